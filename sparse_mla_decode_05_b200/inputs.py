@@ -1,0 +1,238 @@
+"""Seeded synthetic inputs for the sparse-MLA decode step.
+
+This module generates inputs only.  It holds none of the method's
+arithmetic, and both the CUDA library's tests/bench and the fp64 oracle take
+their inputs from it.  All tensors are CPU torch tensors; callers copy them
+to the device.
+
+Workload recipes (shapes, value distributions, index structure):
+
+  c1  B=1,  H=64, q bf16 ~N(0,1); flat bf16 pool [4096, 576] ~N(0,1);
+      top-k = 512 distinct uniform rows.
+  c2  B=16; per-sequence cache lengths uniform in [256, 8192] in one flat
+      bf16 pool (sequence b owns a contiguous run of rows); top-k = 512
+      distinct uniform rows of its own run; when a run is shorter than 512
+      all its rows are used in random order and the list is padded with -1.
+  c3  B=64; 16384 rows per sequence; top-k = 512: 256 distinct rows from the
+      last 1024 (recency-skewed) and 256 distinct uniform rows from the rest,
+      sorted ascending.
+  c4a/c4b  B=1 / B=2; 65536 rows per sequence; top-k = 2048 distinct
+      uniform; q multiplied by 4 (peaky softmax).
+  c5  B=128; paged pool of 16384 pages of 64 rows (1,048,576 rows), fp8
+      e4m3fn codes with one fp32 scale per row (row amax / 448 of an N(0,1)
+      row); each sequence maps 8192 logical positions through a 128-entry
+      page table (a random permutation of all pages); top-k = 2048 distinct
+      uniform logical positions.
+
+scale = 1/sqrt(576) everywhere.  Seeds: workload ci uses seed 1000 + i unless
+one is given.  Normals come from torch's CPU generator (fp32, rounded to
+bf16); index sets from numpy's PCG64 generator.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+H = 64
+D_QK = 576
+D_V = 512
+SCALE = 1.0 / math.sqrt(D_QK)
+
+
+@dataclasses.dataclass
+class Workload:
+    name: str
+    q: torch.Tensor                      # [B, H, D_QK] bfloat16
+    kv: torch.Tensor                     # [N, D_QK] bfloat16, or uint8 (e4m3fn codes)
+    indices: torch.Tensor                # [B, topk] int32, -1 = padding
+    scale: float = SCALE
+    kv_row_scale: torch.Tensor | None = None   # [N] float32 (fp8 pools)
+    page_table: torch.Tensor | None = None     # [B, pages_per_seq] int32
+    page_size: int = 0
+    d_v: int = D_V
+    meta: dict = dataclasses.field(default_factory=dict)
+
+    @property
+    def batch(self) -> int:
+        return self.q.shape[0]
+
+    @property
+    def topk(self) -> int:
+        return self.indices.shape[1]
+
+    @property
+    def kv_format(self) -> str:
+        return "fp8_e4m3_rowscale" if self.kv.dtype == torch.uint8 else "bf16"
+
+    def valid_count(self) -> int:
+        return int((self.indices >= 0).sum())
+
+    # numpy views for the oracle (bit patterns, no arithmetic)
+    def np_q_bits(self) -> np.ndarray:
+        return self.q.view(torch.int16).numpy().view(np.uint16)
+
+    def np_kv(self) -> np.ndarray:
+        if self.kv.dtype == torch.uint8:
+            return self.kv.numpy()
+        return self.kv.view(torch.int16).numpy().view(np.uint16)
+
+
+def _normal_bf16(gen: torch.Generator, shape, mult: float = 1.0,
+                 chunk_rows: int = 65536) -> torch.Tensor:
+    """N(0,1) (times ``mult``) in fp32, rounded to bf16; generated in row
+    chunks to bound host memory."""
+    rows = shape[0]
+    out = torch.empty(shape, dtype=torch.bfloat16)
+    for r0 in range(0, rows, chunk_rows):
+        r1 = min(rows, r0 + chunk_rows)
+        x = torch.randn((r1 - r0,) + tuple(shape[1:]), generator=gen, dtype=torch.float32)
+        if mult != 1.0:
+            x.mul_(mult)
+        out[r0:r1] = x.to(torch.bfloat16)
+    return out
+
+
+def _fp8_rows(gen: torch.Generator, rows: int, chunk_rows: int = 65536):
+    """N(0,1) rows quantised to e4m3fn with a per-row scale amax/448."""
+    codes = torch.empty((rows, D_QK), dtype=torch.uint8)
+    scales = torch.empty((rows,), dtype=torch.float32)
+    for r0 in range(0, rows, chunk_rows):
+        r1 = min(rows, r0 + chunk_rows)
+        x = torch.randn((r1 - r0, D_QK), generator=gen, dtype=torch.float32)
+        s = x.abs().amax(dim=1) / 448.0
+        s = torch.where(s > 0, s, torch.ones_like(s))
+        codes[r0:r1] = (x / s[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        scales[r0:r1] = s
+    return codes, scales
+
+
+def _distinct(rng: np.random.Generator, n: int, k: int) -> np.ndarray:
+    return rng.choice(n, size=k, replace=False).astype(np.int64)
+
+
+def flat_per_seq(B: int, rows_per_seq: int, topk: int, *, seed: int,
+                 q_mult: float = 1.0, index_mode: str = "uniform",
+                 recent_window: int = 1024, name: str = "flat") -> Workload:
+    """Flat bf16 pool of B * rows_per_seq rows; sequence b owns rows
+    [b*R, (b+1)*R).  index_mode "uniform": topk distinct uniform rows;
+    "recency": half from the last ``recent_window`` rows, half uniform from
+    the rest, all distinct, sorted ascending."""
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(gen, (B, H, D_QK), mult=q_mult)
+    kv = _normal_bf16(gen, (B * rows_per_seq, D_QK))
+    idx = np.empty((B, topk), dtype=np.int64)
+    for b in range(B):
+        if index_mode == "uniform":
+            sel = _distinct(rng, rows_per_seq, topk)
+        elif index_mode == "recency":
+            w = min(recent_window, rows_per_seq)
+            n_recent = topk // 2
+            recent = rows_per_seq - w + _distinct(rng, w, n_recent)
+            rest_pool = np.setdiff1d(np.arange(rows_per_seq), recent, assume_unique=True)
+            rest = rest_pool[_distinct(rng, rest_pool.size, topk - n_recent)]
+            sel = np.sort(np.concatenate([recent, rest]))
+        else:
+            raise ValueError(index_mode)
+        idx[b] = sel + b * rows_per_seq
+    return Workload(name=name, q=q, kv=kv, indices=torch.from_numpy(idx.astype(np.int32)),
+                    meta=dict(B=B, rows_per_seq=rows_per_seq, topk=topk, seed=seed,
+                              q_mult=q_mult, index_mode=index_mode))
+
+
+def flat_varlen(B: int, len_lo: int, len_hi: int, topk: int, *, seed: int,
+                name: str = "varlen") -> Workload:
+    """One flat bf16 pool holding B runs with lengths uniform in
+    [len_lo, len_hi]; runs shorter than topk are used whole (shuffled) and
+    padded with -1 at the tail."""
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(len_lo, len_hi + 1, size=B)
+    offs = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    q = _normal_bf16(gen, (B, H, D_QK))
+    kv = _normal_bf16(gen, (int(lens.sum()), D_QK))
+    idx = np.full((B, topk), -1, dtype=np.int64)
+    for b in range(B):
+        if lens[b] >= topk:
+            idx[b] = _distinct(rng, int(lens[b]), topk) + offs[b]
+        else:
+            idx[b, :lens[b]] = rng.permutation(int(lens[b])) + offs[b]
+    return Workload(name=name, q=q, kv=kv, indices=torch.from_numpy(idx.astype(np.int32)),
+                    meta=dict(B=B, lens=lens.tolist(), topk=topk, seed=seed))
+
+
+def paged_fp8(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: int,
+              page_size: int = 64, name: str = "paged_fp8") -> Workload:
+    """Paged fp8 e4m3fn pool with per-row fp32 scales; each sequence's page
+    table row is a slice of one random permutation of all pages."""
+    pps = rows_per_seq // page_size
+    if B * pps > total_pages:
+        raise ValueError("not enough pages for distinct page tables")
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(gen, (B, H, D_QK))
+    codes, scales = _fp8_rows(gen, total_pages * page_size)
+    perm = rng.permutation(total_pages)[: B * pps].reshape(B, pps)
+    idx = np.stack([_distinct(rng, rows_per_seq, topk) for _ in range(B)])
+    return Workload(name=name, q=q, kv=codes, indices=torch.from_numpy(idx.astype(np.int32)),
+                    kv_row_scale=scales, page_table=torch.from_numpy(perm.astype(np.int32)),
+                    page_size=page_size,
+                    meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages,
+                              topk=topk, seed=seed))
+
+
+CONFIG_NAMES = ("c1", "c2", "c3", "c4a", "c4b", "c5")
+
+CONFIG_DESCRIPTIONS = {
+    "c1": "B=1 k=512 flat bf16 pool 4096 rows, uniform distinct",
+    "c2": "B=16 k=512 flat bf16 varlen [256,8192], -1 padded",
+    "c3": "B=64 k=512 flat bf16 16384 rows/seq, recency-skewed sorted",
+    "c4a": "B=1 k=2048 flat bf16 65536 rows/seq, q x4 (split-K stress)",
+    "c4b": "B=2 k=2048 flat bf16 65536 rows/seq, q x4 (split-K stress)",
+    "c5": "B=128 k=2048 paged(64) fp8 e4m3 + row scale, 8192 rows/seq",
+}
+
+
+def make_config(name: str, seed: int | None = None) -> Workload:
+    """The full-size workload ``name`` (one of CONFIG_NAMES)."""
+    base = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005}[name]
+    s = base if seed is None else seed
+    if name == "c1":
+        return flat_per_seq(1, 4096, 512, seed=s, name="c1")
+    if name == "c2":
+        return flat_varlen(16, 256, 8192, 512, seed=s, name="c2")
+    if name == "c3":
+        return flat_per_seq(64, 16384, 512, seed=s, index_mode="recency", name="c3")
+    if name == "c4a":
+        return flat_per_seq(1, 65536, 2048, seed=s, q_mult=4.0, name="c4a")
+    if name == "c4b":
+        return flat_per_seq(2, 65536, 2048, seed=s, q_mult=4.0, name="c4b")
+    if name == "c5":
+        return paged_fp8(128, 8192, 16384, 2048, seed=s, name="c5")
+    raise KeyError(name)
+
+
+def algorithmic_bytes(w: Workload) -> int:
+    """Bytes the step must move at minimum: valid gathered rows (row bytes,
+    plus the 4-byte row scale for fp8 pools), q, out, lse, the index list and
+    the page table.  Padding entries gather nothing."""
+    n_valid = w.valid_count()
+    row = D_QK * (1 if w.kv.dtype == torch.uint8 else 2) + (4 if w.kv_row_scale is not None else 0)
+    B = w.batch
+    b = n_valid * row
+    b += B * H * D_QK * 2          # q
+    b += B * H * w.d_v * 2         # out
+    b += B * H * 4                 # lse
+    b += w.indices.numel() * 4     # indices
+    if w.page_table is not None:
+        b += w.page_table.numel() * 4
+    return int(b)
+
+
+def algorithmic_flops(w: Workload) -> int:
+    """2*H*(d_qk + d_v) flops per valid (sequence, row): the score and the
+    value contractions."""
+    return int(w.valid_count() * 2 * H * (D_QK + w.d_v))
