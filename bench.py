@@ -1,0 +1,383 @@
+"""Benchmark of the sparse-MLA decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+                    [--workload c2] [--no-per-config]
+
+One step = one sparse_mla_decode call (split kernel + combine when the plan
+splits) over one batch of the headline workload, inputs resident in HBM.
+L2 is flushed (a write of 2x the L2 size) before every timed step, outside
+the timed region; each step is timed with CUDA events on the launching
+stream.  With N > 1 (torchrun) every rank runs an independent replica of the
+workload (the op shards over batch with no exchange): weak scaling, time =
+max over ranks.  Rank 0 prints one JSON line.
+
+Keys beyond the base contract:
+  roofline     dominant kernel (the split kernel) vs the measured HBM peak
+  cpu_baseline the fp64 oracle timed on host cores on a bounded sample
+  e2e          same metric through the public call with host (pinned)
+               inputs/outputs copied inside the timed region
+  per_config   microseconds per call and GB/s for every workload, vs roofline
+  clocks       SM clock / throttle reasons sampled during the timed region
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mla_decode_05_b200 import inputs  # noqa: E402
+
+METRIC = "sparse-MLA decode µs/call and gathered-KV HBM GB/s (% of roofline) vs batch"
+HEADLINE = "c2"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        rows = []
+        for line in open(self.file.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- helpers
+def to_dev(w: inputs.Workload, dev):
+    return dict(q=w.q.to(dev), kv=w.kv.to(dev), indices=w.indices.to(dev),
+                kv_row_scale=None if w.kv_row_scale is None else w.kv_row_scale.to(dev),
+                page_table=None if w.page_table is None else w.page_table.to(dev))
+
+
+def roofline_us(w, peak_gbs, peak_tflops):
+    return max(inputs.algorithmic_bytes(w) / (peak_gbs * 1e3), inputs.algorithmic_flops(w) / (peak_tflops * 1e6))
+
+
+class Runner:
+    """Preallocated outputs/workspace for one workload on one device."""
+
+    def __init__(self, w, dev):
+        from sparse_mla_decode_05_b200 import api
+        self.api = api
+        self.w = w
+        self.t = to_dev(w, dev)
+        self.shape = api.shape_for(self.t["q"], self.t["kv"], self.t["indices"], page_table=self.t["page_table"],
+                                   page_size=w.page_size)
+        self.nsplit = api.plan_nsplit(self.shape)
+        ws = api.workspace_size(self.shape)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.out = torch.empty((w.batch, 64, 512), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((w.batch, 64), dtype=torch.float32, device=dev)
+
+    def decode(self, q=None, indices=None):
+        t = self.t
+        return self.api.decode(t["q"] if q is None else q, t["kv"], t["indices"] if indices is None else indices,
+                               self.w.scale, kv_row_scale=t["kv_row_scale"], page_table=t["page_table"],
+                               page_size=self.w.page_size, out=self.out, lse=self.lse, workspace=self.ws)
+
+    def split_only(self):
+        t = self.t
+        return self.api.decode_split(t["q"], t["kv"], t["indices"], self.w.scale, kv_row_scale=t["kv_row_scale"],
+                                     page_table=t["page_table"], page_size=self.w.page_size, out=self.out,
+                                     lse=self.lse, workspace=self.ws)
+
+    def combine_only(self):
+        po, pl = self.api.partial_views(self.ws, self.w.batch, self.nsplit)
+        return self.api.combine(po, pl, out=self.out, lse=self.lse)
+
+    @property
+    def launches_per_step(self):
+        return 1 + (1 if self.nsplit > 1 else 0)
+
+
+def time_device(fn, steps, warmup, flush, stream):
+    """Per-step CUDA-event times (ms) of fn(), L2 flushed before each step."""
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def time_split_breakdown(r: Runner, steps, flush, stream):
+    """Per-step times (ms) of the split kernel and of the combine kernel,
+    each bracketed by events on the launching stream."""
+    sp, cb = [], []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        r.split_only()
+        e1.record(stream)
+        if r.nsplit > 1:
+            r.combine_only()
+        e2.record(stream)
+        sp.append((e0, e1))
+        cb.append((e1, e2))
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in sp], [a.elapsed_time(b) for a, b in cb]
+
+
+def oracle_time(w: inputs.Workload, budget_s: float = 15.0):
+    """fp64 oracle on the host: returns (seconds per full-workload step
+    estimated from a bounded sample, sample description, threads)."""
+    from oracle import sparse_mla_ref as ref
+    B = w.batch
+    args = dict(d_v=w.d_v, kv_format=w.kv_format,
+                kv_row_scale=None if w.kv_row_scale is None else w.kv_row_scale.numpy(),
+                page_table=None if w.page_table is None else w.page_table.numpy(), page_size=w.page_size)
+    qb, kv, idx = w.np_q_bits(), w.np_kv(), w.indices.numpy()
+    done, t_used, reps = 0, 0.0, 0
+    t0 = time.perf_counter()
+    while t_used < budget_s and reps < 1000:
+        for b in range(B):
+            ref.sparse_mla_decode(qb, kv, idx, w.scale, seqs=[b], **args)
+            done += 1
+            t_used = time.perf_counter() - t0
+            if t_used >= budget_s:
+                break
+        reps += 1
+    per_seq = t_used / max(done, 1)
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    return per_seq * B, f"{done} sequences of {w.name} (whole workload = {B} sequences), {t_used:.1f} s", threads
+
+
+# --------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=list(inputs.CONFIG_NAMES))
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--oracle-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peak_gbs, peak_tf, peak_tf_sus, peak_src = load_peaks()
+    w = inputs.make_config(args.workload)
+    alg_bytes = inputs.algorithmic_bytes(w)
+    alg_flops = inputs.algorithmic_flops(w)
+    config = {"workload": f"{args.workload}: {inputs.CONFIG_DESCRIPTIONS[args.workload]}", "batch": w.batch,
+              "topk": w.topk, "heads": 64, "d_qk": 576, "d_v": 512, "kv_dtype": w.kv_format,
+              "paged": w.page_size > 0, "l2": "flushed before every timed step (2x L2 write, untimed)",
+              "parallelism": f"replicas x{args.gpus} (weak)" if args.gpus > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        sec_per_step, sample, threads = oracle_time(w, budget_s=min(args.oracle_budget, 20.0))
+        steps = args.steps
+        val = alg_bytes / sec_per_step / 1e9
+        line = {"metric": METRIC, "value": val, "unit": "GB/s", "impl": "reference", "n_gpus": args.gpus,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": sec_per_step * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": val, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                 "sample": sample},
+                "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    from sparse_mla_decode_05_b200 import api
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    r = Runner(w, dev)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # --- headline: device-resident inputs, whole call
+    barrier()
+    with ClockSampler(local) as clk:
+        t_wall0 = time.perf_counter()
+        times = time_device(r.decode, args.steps, args.warmup, flush, stream)
+        barrier()
+        t_wall = time.perf_counter() - t_wall0
+    clocks = clk.summary()
+    ms = float(np.mean(times))
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    value = alg_bytes * world / (ms * 1e-3) / 1e9
+
+    # --- dominant kernel (split) and combine, each timed on its own
+    sp, cb = time_split_breakdown(r, max(10, args.steps // 2), flush, stream)
+    sp_ms = float(np.mean(sp))
+    cb_ms = float(np.mean(cb)) if r.nsplit > 1 else 0.0
+    achieved = alg_bytes / (sp_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": peak_gbs, "unit": "GB/s", "frac": achieved / peak_gbs,
+            "traffic": None, "kernel": "smla_split_kernel", "peak_source": f"{peak_src} (burst copy)",
+            "split_kernel_us": sp_ms * 1e3, "combine_kernel_us": cb_ms * 1e3, "nsplit": r.nsplit,
+            "roofline_us": roofline_us(w, peak_gbs, peak_tf),
+            "frac_of_step_roofline": roofline_us(w, peak_gbs, peak_tf) / (ms * 1e3),
+            "frac_vs_nominal_8TBps": achieved / 8000.0}
+
+    # --- end to end through the public call: H2D of q + indices (+ page
+    #     table) from pinned memory, decode, D2H of out + lse
+    hq = w.q.pin_memory()
+    hidx = w.indices.pin_memory()
+    hpt = None if w.page_table is None else w.page_table.pin_memory()
+    hout = torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory()
+    hlse = torch.empty(r.lse.shape, dtype=r.lse.dtype).pin_memory()
+    dq = torch.empty_like(r.t["q"])
+    didx = torch.empty_like(r.t["indices"])
+    h2d = hq.numel() * 2 + hidx.numel() * 4 + (0 if hpt is None else hpt.numel() * 4)
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        didx.copy_(hidx, non_blocking=True)
+        if hpt is not None:
+            r.t["page_table"].copy_(hpt, non_blocking=True)
+        r.decode(q=dq, indices=didx)
+        hout.copy_(r.out, non_blocking=True)
+        hlse.copy_(r.lse, non_blocking=True)
+
+    e2e_times = time_device(e2e_step, max(10, args.steps // 2), 3, flush, stream)
+    e2e_ms = float(np.mean(e2e_times))
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e = {"value": alg_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    assert api.device_error() == 0, "device error word set"
+
+    # --- every workload at 1 GPU (rank 0 only)
+    per_config = None
+    if rank == 0 and not args.no_per_config:
+        per_config = []
+        for name in inputs.CONFIG_NAMES:
+            wc = w if name == args.workload else inputs.make_config(name)
+            rc = r if name == args.workload else Runner(wc, dev)
+            tms = time_device(rc.decode, 30, 3, flush, stream)
+            med = float(np.median(tms)) * 1e3
+            p10, p90 = float(np.percentile(tms, 10)) * 1e3, float(np.percentile(tms, 90)) * 1e3
+            spc, _ = time_split_breakdown(rc, 15, flush, stream)
+            ab = inputs.algorithmic_bytes(wc)
+            rl = roofline_us(wc, peak_gbs, peak_tf)
+            per_config.append({"workload": name, "batch": wc.batch, "topk": wc.topk, "nsplit": rc.nsplit,
+                               "us_per_call": med, "p10_us": p10, "p90_us": p90,
+                               "gbs": ab / (med * 1e-6) / 1e9, "roofline_us": rl, "frac_roofline": rl / med,
+                               "split_kernel_us": float(np.median(spc)) * 1e3,
+                               "alg_bytes": ab, "alg_flops": inputs.algorithmic_flops(wc)})
+            if rc is not r:
+                del rc
+                torch.cuda.empty_cache()
+        assert api.device_error() == 0, "device error word set"
+
+    # --- CPU baseline: the oracle on host cores, bounded sample
+    cpu = None
+    if rank == 0 and world == 1:
+        sec, sample, threads = oracle_time(w, budget_s=args.oracle_budget)
+        cpu = {"value": alg_bytes / sec / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "us_per_call": ms * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": config, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": r.launches_per_step * args.steps, "clocks": clocks,
+                "wall_s_timed_region": t_wall, "per_config": per_config}
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

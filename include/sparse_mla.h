@@ -1,0 +1,170 @@
+/*
+ * sparse_mla.h -- C ABI of the B200 (sm_100a) sparse-MLA decode library.
+ *
+ * The operation (one decode step of DeepSeek-style sparse Multi-head Latent
+ * Attention): for every sequence b and head h, one query q[b,h,:] of d_qk =
+ * 576 dims attends over the cache rows named by the sequence's top-k index
+ * list.  Each gathered 576-dim row k_j is the key; its first d_v = 512 dims
+ * are the value.  With s_j = scale * <q[b,h,:], k_j> over the valid entries
+ * (index -1 is padding and takes no part),
+ *
+ *     out[b,h,:] = sum_j softmax(s)_j * k_j[0:512]        (bf16)
+ *     lse[b,h]   = ln sum_j exp(s_j)                        (fp32, natural log)
+ *
+ * A sequence whose list holds no valid entry gets out = 0 and lse = -inf.
+ *
+ * Source pages (by title):
+ *   [Design]  "The MMA Sparse-MLA Decode Kernel: A Deep Dive into AI Inference
+ *              Optimization on Blackwell GPUs" -- "The Agent Reasoning":
+ *              "Kernel Structure Analysis" (query vs. gathered rows, output
+ *              accumulation), "Design Decisions" 1 (head-batched grid: one
+ *              gather shared by the head group), 3 (split-K over top-k),
+ *              6 (bf16 operands, fp32 accumulation), "Edge Case Handling"
+ *              (masked entries), "Validation Strategy" (compare out and LSE).
+ *   [Truth]   "The Moment of Truth: Analyzing a Custom MMA Kernel's
+ *              Performance on Blackwell GPUs" -- "The Split-K Solution:
+ *              Reasoning About the Fix" (partials + combine; grid fixed per
+ *              batch bucket for CUDA-graph capture; scratch deterministic
+ *              per bucket).
+ *   [Pivot]   "The Pivot Point: When a 6.3x Kernel Speedup Reveals the Next
+ *              Bottleneck" -- "The Reasoning: Weighing Two Paths" (split-K
+ *              for the B=1 under-occupancy; combine handles variable NSPLIT).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *    (row-major in the order of the dims given), 16-byte aligned.  The
+ *    library never allocates, frees or retains them.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  Nothing synchronises the host,
+ *    nothing allocates device memory, so a call can be captured in a CUDA
+ *    graph; the grid depends only on the shape (and nsplit).
+ *  - Arguments are validated on the host before any launch.  On a
+ *    validation error nothing is launched and no CUDA call is made.
+ *  - Index values outside [-1, num_kv_rows) (flat) or
+ *    [-1, pages_per_seq * page_size) (paged), and page-table entries outside
+ *    the pool, are caller errors that the kernels do not check.
+ *  - Entry points are thread-safe; they keep no per-call state.
+ */
+#ifndef SPARSE_MLA_H_
+#define SPARSE_MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SMLA_ABI_VERSION 1
+
+typedef enum {
+  SMLA_OK = 0,
+  SMLA_ERR_INVALID_ARG = 1,    /* null / misaligned pointer, bad size        */
+  SMLA_ERR_UNSUPPORTED = 2,    /* shape this build does not implement        */
+  SMLA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
+  SMLA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed       */
+  SMLA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait (see
+                                  sparse_mla_get_device_error)              */
+} smla_status;
+
+typedef enum {
+  SMLA_KV_BF16 = 0,             /* cache rows: bf16 [num_kv_rows, 576]      */
+  SMLA_KV_FP8_E4M3_ROWSCALE = 1 /* cache rows: OCP fp8 e4m3fn codes
+                                   [num_kv_rows, 576] (uint8), and one fp32
+                                   scale per row: value = decode(code)*scale */
+} smla_kv_dtype;
+
+/* Problem description.  num_heads must be 64, d_qk 576, d_v 512. */
+typedef struct {
+  int32_t batch;          /* B >= 1: sequences, one query token each          */
+  int32_t num_heads;      /* H = 64                                            */
+  int32_t d_qk;           /* 576 = 512 latent + 64 rope                        */
+  int32_t d_v;            /* 512: the value is the first 512 dims of the row   */
+  int32_t topk;           /* k >= 1 entries in each index list                 */
+  int32_t kv_dtype;       /* smla_kv_dtype                                     */
+  int64_t num_kv_rows;    /* physical rows in the pool (>= 1)                  */
+  int32_t page_size;      /* 0: flat pool, indices are physical rows.
+                             64: paged pool, indices are logical positions
+                             mapped through page_table                         */
+  int32_t pages_per_seq;  /* width of page_table when page_size > 0           */
+  int32_t nsplit;         /* 0: the planner picks the top-k split; >= 1
+                             forces that many splits (clamped to the number
+                             of 64-entry tiles of the list)                    */
+  int32_t reserved;       /* must be 0                                         */
+} smla_shape;
+
+/* ABI version of the loaded library (SMLA_ABI_VERSION). */
+int32_t sparse_mla_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sparse_mla_status_string(smla_status status);
+
+/* Number of top-k splits the decode will use for `shape` on the current
+ * device: a pure function of (batch, topk, shape->nsplit, SM count), so the
+ * grid is fixed per batch bucket.  Returns 0 if `shape` is invalid. */
+int32_t sparse_mla_plan_nsplit(const smla_shape* shape);
+
+/* Bytes of device workspace sparse_mla_decode needs for `shape` (0 when the
+ * plan uses one split).  Deterministic in the shape, so a workspace sized
+ * once per batch bucket can be reused by every call and every graph replay.
+ * Returns 0 for an invalid shape. */
+size_t sparse_mla_workspace_size(const smla_shape* shape);
+
+/* One decode step (split kernel + combine when the plan splits).
+ *   q            [B, 64, 576] bf16
+ *   kv_cache     [num_kv_rows, 576] bf16, or uint8 e4m3fn codes
+ *   kv_row_scale [num_kv_rows] fp32 for SMLA_KV_FP8_E4M3_ROWSCALE, else NULL
+ *   page_table   [B, pages_per_seq] int32 when page_size > 0, else NULL
+ *   indices      [B, topk] int32, -1 = padding (anywhere in the list)
+ *   scale        softmax scale (e.g. 1/sqrt(576))
+ *   out          [B, 64, 512] bf16   (written)
+ *   lse          [B, 64] fp32        (written; natural log, scale included)
+ *   workspace    device scratch of >= sparse_mla_workspace_size() bytes,
+ *                256-byte aligned; may be NULL when that size is 0.  Its
+ *                contents need no initialisation and are garbage afterwards.
+ * Two calls that share a workspace must be ordered on the GPU (same stream
+ * or event-ordered).  Returns SMLA_OK after launching. */
+smla_status sparse_mla_decode(const smla_shape* shape, const void* q, const void* kv_cache,
+                              const float* kv_row_scale, const int32_t* page_table,
+                              const int32_t* indices, float scale, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* The split kernel alone: the hot loop of sparse_mla_decode.
+ * With nsplit == 1 it writes out/lse directly (workspace unused).  With
+ * nsplit > 1 it writes per-split partial results into the workspace:
+ *   partial_o   = workspace                      [B, nsplit, 64, 512] fp32,
+ *                 each split's output normalised by its own softmax sum
+ *                 (0 when the split holds no valid entry)
+ *   partial_lse = workspace + B*nsplit*64*512*4  [B, nsplit, 64] fp32
+ *                 (that split's log-sum-exp, -inf when empty)
+ * and out/lse are not touched (sparse_mla_combine finishes them).  *nsplit_out
+ * (may be NULL) receives the split count used. */
+smla_status sparse_mla_decode_split(const smla_shape* shape, const void* q, const void* kv_cache,
+                                    const float* kv_row_scale, const int32_t* page_table,
+                                    const int32_t* indices, float scale, void* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, int32_t* nsplit_out,
+                                    void* stream);
+
+/* Log-sum-exp combine of per-split partials ([Truth] "The Split-K Solution").
+ *   partial_o   [B, nsplit, H, d_v] fp32 (normalised per split)
+ *   partial_lse [B, nsplit, H] fp32 (-inf for an empty split)
+ *   out         [B, H, d_v] bf16, lse [B, H] fp32
+ * With L = ln sum_s exp(lse_s): out = sum_s exp(lse_s - L) * o_s, lse = L;
+ * every split empty gives out = 0, lse = -inf.  Requires H == 64,
+ * d_v == 512, 1 <= nsplit <= 4096. */
+smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, int32_t nsplit,
+                               const float* partial_o, const float* partial_lse, void* out,
+                               float* lse, void* stream);
+
+/* Reads and clears the library's device error word on the current device
+ * (a synchronous device-to-host copy: call it outside timed or captured
+ * regions).  *code receives the raw word (0 = no error; bit 0: a kernel gave
+ * up waiting on a pipeline barrier).  Returns SMLA_ERR_DEVICE_TIMEOUT if
+ * the word was non-zero, SMLA_OK if zero, SMLA_ERR_CUDA on a copy failure. */
+smla_status sparse_mla_get_device_error(uint32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_MLA_H_ */

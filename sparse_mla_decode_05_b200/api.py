@@ -1,0 +1,191 @@
+"""Thin Python binding over the C ABI in include/sparse_mla.h.
+
+Argument marshalling only: every step of the decode runs in the CUDA
+library.  Torch tensors supply device pointers and the current stream.
+There is no fallback: if the shared library is missing this module raises
+on import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsparse_mla.so")
+
+H, D_QK, D_V, TILE = 64, 576, 512, 64
+KV_BF16, KV_FP8_E4M3_ROWSCALE = 0, 1
+
+STATUS = {0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARG", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_WORKSPACE",
+          4: "SMLA_ERR_CUDA", 5: "SMLA_ERR_DEVICE_TIMEOUT"}
+
+
+class SmlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class SmlaShape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("d_qk", ctypes.c_int32),
+        ("d_v", ctypes.c_int32), ("topk", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+        ("num_kv_rows", ctypes.c_int64), ("page_size", ctypes.c_int32),
+        ("pages_per_seq", ctypes.c_int32), ("nsplit", ctypes.c_int32), ("reserved", ctypes.c_int32),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_mla_decode_05_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, SZ, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.c_float
+    SP = ctypes.POINTER(SmlaShape)
+    lib.sparse_mla_abi_version.restype = I32
+    lib.sparse_mla_status_string.restype = ctypes.c_char_p
+    lib.sparse_mla_status_string.argtypes = [I32]
+    lib.sparse_mla_plan_nsplit.restype = I32
+    lib.sparse_mla_plan_nsplit.argtypes = [SP]
+    lib.sparse_mla_workspace_size.restype = SZ
+    lib.sparse_mla_workspace_size.argtypes = [SP]
+    lib.sparse_mla_decode.restype = I32
+    lib.sparse_mla_decode.argtypes = [SP, P, P, P, P, P, F32, P, P, P, SZ, P]
+    lib.sparse_mla_decode_split.restype = I32
+    lib.sparse_mla_decode_split.argtypes = [SP, P, P, P, P, P, F32, P, P, P, SZ,
+                                            ctypes.POINTER(I32), P]
+    lib.sparse_mla_combine.restype = I32
+    lib.sparse_mla_combine.argtypes = [I32, I32, I32, I32, P, P, P, P, P]
+    lib.sparse_mla_get_device_error.restype = I32
+    lib.sparse_mla_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    return lib
+
+
+lib = _load()
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def make_shape(batch: int, topk: int, num_kv_rows: int, *, fp8: bool = False, page_size: int = 0,
+               pages_per_seq: int = 0, nsplit: int = 0) -> SmlaShape:
+    return SmlaShape(batch, H, D_QK, D_V, topk, KV_FP8_E4M3_ROWSCALE if fp8 else KV_BF16,
+                     num_kv_rows, page_size, pages_per_seq, nsplit, 0)
+
+
+def shape_for(q, kv, indices, *, page_table=None, page_size: int = 0, nsplit: int = 0) -> SmlaShape:
+    return make_shape(q.shape[0], indices.shape[1], kv.shape[0], fp8=(kv.dtype == torch.uint8),
+                      page_size=page_size,
+                      pages_per_seq=0 if page_table is None else page_table.shape[1], nsplit=nsplit)
+
+
+def plan_nsplit(shape: SmlaShape) -> int:
+    return lib.sparse_mla_plan_nsplit(ctypes.byref(shape))
+
+
+def workspace_size(shape: SmlaShape) -> int:
+    return lib.sparse_mla_workspace_size(ctypes.byref(shape))
+
+
+def _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size):
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[1:] != (H, D_QK):
+        raise ValueError("q must be bf16 [B, 64, 576]")
+    if kv.dim() != 2 or kv.shape[1] != D_QK or kv.dtype not in (torch.bfloat16, torch.uint8):
+        raise ValueError("kv must be [N, 576] bf16 or uint8 (fp8 e4m3fn codes)")
+    if indices.dtype != torch.int32 or indices.dim() != 2 or indices.shape[0] != q.shape[0]:
+        raise ValueError("indices must be int32 [B, topk]")
+    if kv.dtype == torch.uint8 and (kv_row_scale is None or kv_row_scale.dtype != torch.float32):
+        raise ValueError("fp8 cache needs float32 kv_row_scale [N]")
+    if page_size and (page_table is None or page_table.dtype != torch.int32):
+        raise ValueError("paged cache needs int32 page_table [B, pages_per_seq]")
+    for t in (q, kv, indices, kv_row_scale, page_table):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+
+
+def decode(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=None, page_size: int = 0,
+           nsplit: int = 0, out=None, lse=None, workspace=None):
+    """out [B,64,512] bf16, lse [B,64] fp32 = sparse-MLA decode (one call to
+    sparse_mla_decode).  Allocates out / lse / workspace with torch when not
+    given."""
+    _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size)
+    shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
+    dev = q.device
+    if out is None:
+        out = torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
+    ws_bytes = workspace_size(shape)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = lib.sparse_mla_decode(ctypes.byref(shape), _ptr(q), _ptr(kv), _ptr(kv_row_scale),
+                               _ptr(page_table), _ptr(indices), float(scale), _ptr(out), _ptr(lse),
+                               _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                               _stream(dev))
+    if st != 0:
+        raise SmlaError(st, "sparse_mla_decode")
+    return out, lse
+
+
+def decode_split(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=None,
+                 page_size: int = 0, nsplit: int = 0, out=None, lse=None, workspace=None):
+    """The split kernel alone.  Returns (nsplit, out, lse, workspace); with
+    nsplit > 1 the partial results are in the workspace (see the header)."""
+    _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size)
+    shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
+    dev = q.device
+    if out is None:
+        out = torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
+    ws_bytes = workspace_size(shape)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    n = ctypes.c_int32(0)
+    st = lib.sparse_mla_decode_split(ctypes.byref(shape), _ptr(q), _ptr(kv), _ptr(kv_row_scale),
+                                     _ptr(page_table), _ptr(indices), float(scale), _ptr(out),
+                                     _ptr(lse), _ptr(workspace),
+                                     0 if workspace is None else workspace.numel(), ctypes.byref(n),
+                                     _stream(dev))
+    if st != 0:
+        raise SmlaError(st, "sparse_mla_decode_split")
+    return n.value, out, lse, workspace
+
+
+def partial_views(workspace, batch: int, nsplit: int):
+    """(partial_o [B, nsplit, 64, 512] fp32, partial_lse [B, nsplit, 64] fp32)
+    views of a split workspace."""
+    n_o = batch * nsplit * H * D_V
+    f = workspace.view(torch.float32)
+    return f[:n_o].view(batch, nsplit, H, D_V), f[n_o:n_o + batch * nsplit * H].view(batch, nsplit, H)
+
+
+def combine(partial_o, partial_lse, out=None, lse=None):
+    """out, lse = log-sum-exp combine of per-split partials (sparse_mla_combine)."""
+    B, n, h, dv = partial_o.shape
+    dev = partial_o.device
+    if out is None:
+        out = torch.empty((B, h, dv), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, h), dtype=torch.float32, device=dev)
+    st = lib.sparse_mla_combine(B, h, dv, n, _ptr(partial_o), _ptr(partial_lse), _ptr(out), _ptr(lse),
+                                _stream(dev))
+    if st != 0:
+        raise SmlaError(st, "sparse_mla_combine")
+    return out, lse
+
+
+def device_error() -> int:
+    """Reads and clears the device error word (synchronous)."""
+    code = ctypes.c_uint32(0)
+    st = lib.sparse_mla_get_device_error(ctypes.byref(code))
+    if st not in (0, 5):
+        raise SmlaError(st, "sparse_mla_get_device_error")
+    return code.value

@@ -1,0 +1,129 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry
+point include/sparse_mla.h declares, and rejects bad arguments on the host
+before making any CUDA call."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparse_mla.h")
+
+
+def _ensure_built():
+    from sparse_mla_decode_05_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build_library()
+
+
+_ensure_built()
+from sparse_mla_decode_05_b200 import api  # noqa: E402
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sparse_mla_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("sparse_mla_decode", "sparse_mla_decode_split", "sparse_mla_combine",
+                 "sparse_mla_workspace_size", "sparse_mla_plan_nsplit", "sparse_mla_status_string",
+                 "sparse_mla_abi_version", "sparse_mla_get_device_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(api.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_and_status_strings():
+    assert api.lib.sparse_mla_abi_version() == 1
+    for code, name in api.STATUS.items():
+        assert api.lib.sparse_mla_status_string(code).decode() == name
+    assert api.lib.sparse_mla_status_string(99).decode() == "SMLA_ERR_UNKNOWN"
+
+
+def test_struct_layout_matches_header():
+    assert ctypes.sizeof(api.SmlaShape) == 48
+    assert api.SmlaShape.num_kv_rows.offset == 24
+
+
+def _decode(shape, q=16, kv=16, rs=None, pt=None, idx=16, scale=0.04, out=16, lse=16, ws=None, nbytes=0):
+    return api.lib.sparse_mla_decode(ctypes.byref(shape) if shape is not None else None, q, kv, rs, pt, idx,
+                                     scale, out, lse, ws, nbytes, None)
+
+
+GOOD = dict(batch=2, topk=100, num_kv_rows=1000)
+
+
+def shape(**kw):
+    d = dict(GOOD)
+    d.update(kw)
+    s = api.make_shape(d.pop("batch"), d.pop("topk"), d.pop("num_kv_rows"), fp8=d.pop("fp8", False),
+                       page_size=d.pop("page_size", 0), pages_per_seq=d.pop("pages_per_seq", 0),
+                       nsplit=d.pop("nsplit", 0))
+    for k, v in d.items():
+        setattr(s, k, v)
+    return s
+
+
+INVALID, UNSUPPORTED = 1, 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), INVALID), (dict(batch=70000), INVALID), (dict(topk=0), INVALID),
+    (dict(num_kv_rows=0), INVALID), (dict(nsplit=-1), INVALID), (dict(reserved=1), INVALID),
+    (dict(num_heads=32), UNSUPPORTED), (dict(d_qk=512), UNSUPPORTED), (dict(d_v=576), UNSUPPORTED),
+    (dict(kv_dtype=7), UNSUPPORTED), (dict(page_size=32, pages_per_seq=4), UNSUPPORTED),
+    (dict(page_size=64, pages_per_seq=0), INVALID),
+])
+def test_bad_shapes_rejected_without_cuda(kw, code):
+    assert _decode(shape(**kw)) == code
+    assert api.lib.sparse_mla_workspace_size(ctypes.byref(shape(**kw))) == 0
+    assert api.lib.sparse_mla_plan_nsplit(ctypes.byref(shape(**kw))) == 0
+
+
+def test_null_and_misaligned_pointers_rejected():
+    s = shape()
+    assert _decode(None) == INVALID
+    assert _decode(s, q=None) == INVALID
+    assert _decode(s, kv=None) == INVALID
+    assert _decode(s, idx=None) == INVALID
+    assert _decode(s, out=None) == INVALID
+    assert _decode(s, lse=None) == INVALID
+    assert _decode(s, q=24) == INVALID            # not 16-byte aligned
+    assert _decode(s, kv=8) == INVALID
+    assert _decode(s, out=40) == INVALID
+    assert _decode(s, idx=18) == INVALID           # not 4-byte aligned
+    assert _decode(s, scale=math.nan) == INVALID
+    assert _decode(s, scale=math.inf) == INVALID
+    assert _decode(shape(fp8=True)) == INVALID      # fp8 without row scales
+    assert _decode(shape(page_size=64, pages_per_seq=3)) == INVALID   # paged without a table
+
+
+def test_combine_argument_checks():
+    c = api.lib.sparse_mla_combine
+    assert c(0, 64, 512, 2, 16, 16, 16, 16, None) == INVALID
+    assert c(1, 64, 512, 0, 16, 16, 16, 16, None) == INVALID
+    assert c(1, 64, 512, 5000, 16, 16, 16, 16, None) == INVALID
+    assert c(1, 32, 512, 2, 16, 16, 16, 16, None) == UNSUPPORTED
+    assert c(1, 64, 256, 2, 16, 16, 16, 16, None) == UNSUPPORTED
+    assert c(1, 64, 512, 2, None, 16, 16, 16, None) == INVALID
+    assert c(1, 64, 512, 2, 8, 16, 16, 16, None) == INVALID
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 64, 576, dtype=torch.bfloat16)
+    kv = torch.zeros(10, 576, dtype=torch.bfloat16)
+    idx = torch.zeros(1, 4, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        api.decode(q, kv, idx, 0.04)
+    with pytest.raises(ValueError):
+        api.decode(q[:, :32], kv, idx, 0.04)
