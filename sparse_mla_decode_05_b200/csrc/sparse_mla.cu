@@ -537,7 +537,11 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     const int h = 16 * warp + (lane & 15);   // head row of this thread
     const int half = lane >> 4;              // tokens [32*half, 32*half+32)
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
+    // l_run: sum of the probabilities as fp32 (gives lse); l_pv: the same sum
+    // of the bf16-rounded probabilities the PV MMA used (normalises out, so
+    // the output weights sum to one exactly).  fp8 rows fold the row scale
+    // into P, so there l_pv = l_run.
+    float m_run = -INFINITY, l_run = 0.f, l_pv = 0.f;
     bool aborted = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1;
@@ -569,7 +573,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       const float m_use = need ? m_new : m_run;
       const float alpha = need ? ex2(m_run - m_use) : 1.f;
       uint32_t pk[16];
-      float lsum = 0.f;
+      float lsum = 0.f, lsum_pv = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; j += 2) {
         const float p0 = s[j] == -INFINITY ? 0.f : ex2(s[j] - m_use);
@@ -580,7 +584,8 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         } else {
           const uint32_t w = pack_bf16x2(p0, p1);
           pk[j / 2] = w;
-          lsum += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+          lsum += p0 + p1;
+          lsum_pv += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
         }
       }
       // P buffer and O are free once PV(i-1) has completed
@@ -606,6 +611,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         tmem_wait_st();
       }
       l_run = l_run * alpha + lsum;
+      l_pv = kFp8 ? l_run : l_pv * alpha + lsum_pv;
       m_run = m_use;
       const uint32_t prow = sbase + kSmemP;
 #pragma unroll
@@ -625,9 +631,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     }
     if (!aborted) {
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       const bool any = l_tot > 0.f;
       if (half == 0) {
-        s_invl[h] = any ? 1.f / l_tot : 0.f;
+        s_invl[h] = any ? 1.f / l_nrm : 0.f;
         s_lse[h] = any ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
       }
       named_bar_sync(2, 128);

@@ -38,22 +38,19 @@ def oracle(w: inputs.Workload, seqs=None):
 
 
 def compare(out_gpu, lse_gpu, out_ref, lse_ref, seqs=None):
-    """Returns (max abs out error, max lse rel error, max bf16-ulp distance
-    from bf16(oracle)) over the selected sequences."""
+    """Returns (max abs out error, max lse rel error, max error in bf16 ulps)
+    over the selected sequences."""
     o = out_gpu.float().cpu().numpy().astype(np.float64)
     l = lse_gpu.cpu().numpy().astype(np.float64)
     if seqs is not None:
         o, l, out_ref, lse_ref = o[seqs], l[seqs], out_ref[seqs], lse_ref[seqs]
     err = float(np.max(np.abs(o - out_ref))) if o.size else 0.0
     lerr = float(np.max(ref.lse_rel_err(l, lse_ref))) if l.size else 0.0
-    want_bits = ref.f64_to_bf16_bits_rne(out_ref).astype(np.int64)
-    got_bits = out_gpu.cpu().view(torch.int16).numpy().astype(np.int64) & 0xFFFF
-    if seqs is not None:
-        got_bits = got_bits[seqs]
-    # ulp distance on the sign-magnitude bit line
-    def line(b):
-        return np.where(b & 0x8000, -(b & 0x7FFF), b & 0x7FFF)
-    ulps = int(np.max(np.abs(line(got_bits) - line(want_bits)))) if got_bits.size else 0
+    # error in units of the bf16 ulp at |ref| (|ref| floored at 2^-6 so that
+    # values near zero do not blow the unit up)
+    mag = np.maximum(np.abs(out_ref), 2.0 ** -6)
+    ulp = 2.0 ** (np.floor(np.log2(mag)) - 7)
+    ulps = float(np.max(np.abs(o - out_ref) / ulp)) if o.size else 0.0
     return err, lerr, ulps
 
 

@@ -39,7 +39,7 @@ def test_full_config_parity(name):
     out_ref, lse_ref = oracle(w)
     err, lerr, ulps = assert_parity(out, lse, out_ref, lse_ref, tag=name)
     print(f"{name}: nsplit={api().plan_nsplit(api().shape_for(d.q, d.kv, d.indices, page_table=d.page_table, page_size=w.page_size))} "
-          f"max|dout|={err:.3e} lse_rel={lerr:.3e} max_ulps={ulps}")
+          f"max|dout|={err:.3e} lse_rel={lerr:.3e} max_err_ulps={ulps:.2f}")
 
 
 @pytest.mark.parametrize("name", ["c2", "c4b"])
@@ -272,3 +272,23 @@ def test_cuda_graph_replay_bit_identical(name):
     assert torch.equal(out.view(torch.int16), eager_out.view(torch.int16))
     assert torch.equal(lse, eager_lse)
     del g
+
+
+def test_workspace_checks():
+    w = inputs.flat_per_seq(2, 1000, 300, seed=1)
+    d = Dev(w)
+    a = api()
+    shape = a.shape_for(d.q, d.kv, d.indices, nsplit=3)
+    need = a.workspace_size(shape)
+    assert need > 0 and need % 256 == 0 and a.plan_nsplit(shape) == 3
+    small = torch.empty(need - 256, dtype=torch.uint8, device="cuda:0")
+    with pytest.raises(a.SmlaError) as e:
+        d.run(nsplit=3, workspace=small)
+    assert e.value.code == 3
+    big = torch.empty(need + 512, dtype=torch.uint8, device="cuda:0")
+    with pytest.raises(a.SmlaError) as e:
+        d.run(nsplit=3, workspace=big[16:])          # not 256-byte aligned
+    assert e.value.code == 3
+    one = a.shape_for(d.q, d.kv, d.indices, nsplit=1)
+    assert a.workspace_size(one) == 0
+    d.run(nsplit=1, workspace=None)                  # no workspace needed
