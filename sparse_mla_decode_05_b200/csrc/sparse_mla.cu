@@ -42,11 +42,13 @@
 // records an error bit in a device word, drains its own copies and MMAs,
 // frees TMEM and exits.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 #include <math.h>
+#include <string.h>
 
 #include "sparse_mla.h"
 
@@ -63,26 +65,37 @@ constexpr int kTileBytes = kAtoms * kAtomBytes;     // 73,728
 constexpr int kRowBytesBf16 = kDqk * 2;             // 1152
 constexpr int kRowBytesFp8 = kDqk;                  // 576
 
-// shared memory map (offsets from a 1024-aligned base)
+// shared memory map (offsets from the 1024-aligned dynamic shared base)
 constexpr int kSmemQ = 0;                           // Q   [9 atoms][64 heads][128 B]
 constexpr int kSmemKV = kSmemQ + kTileBytes;        // KV  [2 stages][9 atoms][64 tok][128 B]
 constexpr int kSmemP = kSmemKV + 2 * kTileBytes;    // P   [64 heads][64 tok] bf16 (K-major)
 constexpr int kSmemAux = kSmemP + 64 * 128;
-constexpr int kNumBars = 12;
-constexpr int kAuxBars = kSmemAux;                  // 12 mbarriers
-constexpr int kAuxTmem = kAuxBars + 8 * kNumBars;   // TMEM base address (4 B)
-constexpr int kAuxRow = kAuxTmem + 16;              // int  [2][64] physical row or -1
-constexpr int kAuxRsc = kAuxRow + 2 * 64 * 4;       // f32  [2][64] fp8 row scales
-constexpr int kAuxAlpha = kAuxRsc + 2 * 64 * 4;     // f32  [64] rescale factors
-constexpr int kAuxInvl = kAuxAlpha + 64 * 4;        // f32  [64] 1/l
-constexpr int kAuxLse = kAuxInvl + 64 * 4;          // f32  [64] lse
-constexpr int kAuxEnd = kAuxLse + 64 * 4;
-constexpr int kSmemBytes = kAuxEnd + 1024;          // + alignment slack
-static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
-
+constexpr int kRing = 4;                            // resolved-row ring depth (tiles)
 // barrier indices
-constexpr int BAR_Q = 0, BAR_KVF = 1, BAR_KVE = 3, BAR_SF = 5, BAR_SE = 7, BAR_PF = 9,
-              BAR_PVD = 10, BAR_FIN = 11;
+constexpr int BAR_Q = 0;
+constexpr int BAR_KVF = 1;                          // [2 stages][9 atoms]
+constexpr int BAR_KVE = BAR_KVF + 2 * kAtoms;       // [2]
+constexpr int BAR_SF = BAR_KVE + 2;                 // [2]
+constexpr int BAR_SE = BAR_SF + 2;                  // [2]
+constexpr int BAR_PF = BAR_SE + 2;
+constexpr int BAR_PVD = BAR_PF + 1;
+constexpr int BAR_FIN = BAR_PVD + 1;
+constexpr int BAR_FIN2 = BAR_FIN + 1;
+constexpr int BAR_IXF = BAR_FIN2 + 1;               // [kRing]
+constexpr int BAR_IXE = BAR_IXF + kRing;            // [kRing]
+constexpr int kNumBars = BAR_IXE + kRing;
+constexpr int kAuxBars = kSmemAux;
+constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
+constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
+constexpr int kAuxRsc = kAuxRow + kRing * 64 * 4;   // f32  [kRing][64] fp8 row scales
+constexpr int kAuxAlpha = kAuxRsc + kRing * 64 * 4; // f32  [64] rescale factors
+constexpr int kAuxEnd = kAuxAlpha + 64 * 4;
+constexpr int kSmemBytes = kAuxEnd;
+// epilogue scratch inside the (then idle) P buffer
+constexpr int kEpiInvl = kSmemP;                    // f32 [64] 1/l
+constexpr int kEpiLse = kSmemP + 256;               // f32 [64] lse
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
+static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxAlpha % 16 == 0, "aux arrays are read as 16-byte vectors");
 
 // TMEM columns (512 allocated): O^T chunks at 0..255, S buffers at 256 and 320
 constexpr uint32_t kTmemCols = 512;
@@ -102,16 +115,22 @@ constexpr uint32_t make_idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
 constexpr uint32_t kIdescS = make_idesc(64, 64, false, false);    // S  = Q K^T
 constexpr uint32_t kIdescPV = make_idesc(128, 64, true, false);   // O^T = V^T P^T
 
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Bounded waits give up after this many SM clock cycles (about 2 s).
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
+// warps 0-3 softmax/epilogue, 4 S-MMA issuer (+ TMEM allocator), 5 PV-MMA
+// issuer, 6 index resolver, 7.. loaders (bf16 rows: four warps issuing
+// 16-byte cp.async; fp8 rows: eight warps that load, convert and store)
+constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kWarpLoad0 = 7;
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kProdWarps = kFp8 ? 8 : 4;
-  static constexpr int kProdThreads = kProdWarps * 32;
-  static constexpr int kThreads = (4 + 1 + kProdWarps) * 32;
+  static constexpr int kLoadWarps = kFp8 ? 8 : 4;
+  static constexpr int kLoadThreads = kLoadWarps * 32;
+  static constexpr int kThreads = (kWarpLoad0 + kLoadWarps) * 32;
 };
 
 struct SplitParams {
+  CUtensorMap tmap_q;          // q as [B*64, 576]: box 64 x 64, 128B swizzle
   const uint8_t* q;            // [B, 64, 576] bf16
   const uint8_t* kv;           // rows of 1152 B (bf16) or 576 B (fp8 codes)
   const float* kv_row_scale;   // [N] (fp8)
@@ -166,12 +185,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // Bounded wait: false (and an error bit) if the phase did not complete in time.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       atomicOr(&g_error_word, 1u);
       return false;
     }
@@ -261,14 +280,32 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
 }
-// D[tmem] (+)= A[smem desc] . B[smem desc]
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
+// Warp-uniform MMA issue: the whole warp computes the (uniform) operands and
+// one elected lane executes the instruction.  D[tmem] = A . B ("set", first K
+// step) or D[tmem] += A . B ("acc").
+__device__ __forceinline__ void mma_set_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.u32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.u32 p, 0, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_acc_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.eq.u32 p, 0, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
+__device__ __forceinline__ void commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -342,12 +379,44 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
 }
 
 // ============================================================ split kernel
+#ifdef SMLA_TRACE
+// Development-only timeline probe (compiled only with -DSMLA_TRACE): the
+// global timer at fixed pipeline events of the first 256 CTAs.
+__device__ unsigned long long g_trace[256 * 64];
+#define SMLA_TRACE_EV(ev)                                                          \
+  do {                                                                             \
+    const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                          \
+    if (cta_ < 256 && (ev) < 64) g_trace[cta_ * 64 + (ev)] = globaltimer_ns();     \
+  } while (0)
+#else
+#define SMLA_TRACE_EV(ev) do { } while (0)
+#endif
+
+__device__ __forceinline__ void bulk_store_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     smla_split_kernel(const __grid_constant__ SplitParams p) {
-  constexpr int kProd = Cfg<kFp8>::kProdThreads;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int kLoad = Cfg<kFp8>::kLoadThreads;
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bars = sbase + kAuxBars;
   auto BAR = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
@@ -362,26 +431,42 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   const int tok_begin = t_begin * kTile;
   const int tok_end = min(t_end * kTile, p.topk);
 
+  // The swizzled operand layouts need a 1024-byte aligned base; the dynamic
+  // shared window starts there when the kernel has no static shared memory.
+  if (sbase & 1023u) {
+    if (threadIdx.x == 0) atomicOr(&g_error_word, 2u);
+    return;
+  }
+  SMLA_TRACE_EV(0);
+
   int* s_row = reinterpret_cast<int*>(smem + kAuxRow);
   float* s_rsc = reinterpret_cast<float*>(smem + kAuxRsc);
   float* s_alpha = reinterpret_cast<float*>(smem + kAuxAlpha);
-  float* s_invl = reinterpret_cast<float*>(smem + kAuxInvl);
-  float* s_lse = reinterpret_cast<float*>(smem + kAuxLse);
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(BAR_Q), kProd);
+    mbar_init(BAR(BAR_Q), 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(BAR(BAR_KVF + s), kFp8 ? kProd : 2 * kProd);
+      // tile barrier (the first of the stage's atom slots is used): bf16 ->
+      // every loader thread's asynchronous arrival; fp8 -> one per loader warp
+      mbar_init(BAR(BAR_KVF + s * kAtoms), kFp8 ? kLoad / 32 : kLoad);
       mbar_init(BAR(BAR_KVE + s), 1);
       mbar_init(BAR(BAR_SF + s), 1);
-      mbar_init(BAR(BAR_SE + s), 128);
+      mbar_init(BAR(BAR_SE + s), 4);      // one arrival per softmax warp
     }
-    mbar_init(BAR(BAR_PF), 128);
+    mbar_init(BAR(BAR_PF), 4);
     mbar_init(BAR(BAR_PVD), 1);
     mbar_init(BAR(BAR_FIN), 1);
+    mbar_init(BAR(BAR_FIN2), 1);
+    // Arrivals are per warp (a warp synchronises, then one lane arrives):
+    // mbarrier arrivals are serialised, so hundreds of per-thread arrivals
+    // per tile would sit on the critical path.
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(BAR(BAR_IXF + r), 1);
+      mbar_init(BAR(BAR_IXE + r), kLoad / 32 + 4);  // loader warps + softmax warps
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 4) {
+  if (warp == kWarpS) {
     tmem_alloc(sbase + kAuxTmem, kTmemCols);
     tmem_relinquish();
   }
@@ -389,149 +474,206 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kAuxTmem);
+  SMLA_TRACE_EV(1);
 
-  if (warp >= 5) {
-    // ------------------------------------------------------------ producers
-    const int ptid = threadIdx.x - 160;
-    {  // the 64 x 576 query, once, into the 128B-swizzled K-major layout
-      const uint8_t* qsrc = p.q + (size_t)b * kH * kRowBytesBf16;
-      for (int c = ptid; c < kH * 72; c += kProd) {
-        const int h = c / 72, ch = c - h * 72;
-        const uint32_t dst = sbase + kSmemQ + (ch >> 3) * kAtomBytes + sw128_off(h, ch & 7);
-        cp_async_16(dst, qsrc + (size_t)h * kRowBytesBf16 + ch * 16, 16);
+  if (warp == kWarpIdx) {
+    // ------------------------------------------------------------ index warp
+    // Resolves each tile's 64 entries to physical rows (and fp8 row scales)
+    // into a kRing-deep ring, running ahead of the loaders.  Loads are
+    // software-pipelined: index of tile t+2, page entry of t+1, scale of t.
+    auto idx_at = [&](int t, int j) -> int {
+      const int pos = tok_begin + t * kTile + j;
+      return (t < ntiles && pos < tok_end) ? __ldg(p.indices + (size_t)b * p.topk + pos) : -1;
+    };
+    auto row_of = [&](int idx) -> int {
+      if (idx < 0) return -1;
+      if (!p.page_size) return idx;
+      return __ldg(p.page_table + (size_t)b * p.pages_per_seq + idx / p.page_size) * p.page_size +
+             idx % p.page_size;
+    };
+    int ia0 = idx_at(0, lane), ia1 = idx_at(0, lane + 32);
+    int ib0 = idx_at(1, lane), ib1 = idx_at(1, lane + 32);
+    int r0 = row_of(ia0), r1 = row_of(ia1);
+    for (int t = 0; t < ntiles; ++t) {
+      const int rs = t % kRing;
+      float c0 = 0.f, c1 = 0.f;
+      if (kFp8) {
+        c0 = r0 >= 0 ? __ldg(p.kv_row_scale + r0) : 0.f;
+        c1 = r1 >= 0 ? __ldg(p.kv_row_scale + r1) : 0.f;
       }
-      cp_async_mbar_arrive_noinc(BAR(BAR_Q));
+      const int n0 = row_of(ib0), n1 = row_of(ib1);
+      // rows of tile t+1 are known now: start pulling them into L2
+      {
+        constexpr uint32_t kRowBytes = kFp8 ? kRowBytesFp8 : kRowBytesBf16;
+        if (n0 >= 0) prefetch_l2(p.kv + (size_t)n0 * kRowBytes, kRowBytes);
+        if (n1 >= 0) prefetch_l2(p.kv + (size_t)n1 * kRowBytes, kRowBytes);
+      }
+      const int ic0 = idx_at(t + 2, lane), ic1 = idx_at(t + 2, lane + 32);
+      if (t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1)) break;
+      s_row[rs * 64 + lane] = r0;
+      s_row[rs * 64 + lane + 32] = r1;
+      if (kFp8) {
+        s_rsc[rs * 64 + lane] = c0;
+        s_rsc[rs * 64 + lane + 32] = c1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_IXF + rs));
+      r0 = n0;
+      r1 = n1;
+      ib0 = ic0;
+      ib1 = ic1;
+    }
+  } else if (warp >= kWarpLoad0) {
+    // ------------------------------------------------------------ loaders
+    const int lt = threadIdx.x - 32 * kWarpLoad0;  // 0 .. kLoad-1
+    if (lt == 0) {  // the 64 x 576 query: nine 64 x 64 TMA boxes, 128B-swizzled K-major
+      mbar_arrive_expect_tx(BAR(BAR_Q), (uint32_t)kTileBytes);
+      for (int a = 0; a < kAtoms; ++a)
+        tma_load_2d(sbase + kSmemQ + a * kAtomBytes, &p.tmap_q, a * 64, b * kH, BAR(BAR_Q));
     }
     for (int t = 0; t < ntiles; ++t) {
-      const int slot = t & 1;
-      bool fail = false;
-      if (t >= 2) fail = !mbar_wait(BAR(BAR_KVE + slot), ((t >> 1) - 1) & 1);
-      if (group_any(fail, 1, kProd)) break;
-      if (ptid < kTile) {  // index -> physical row (or -1)
-        const int pos = tok_begin + t * kTile + ptid;
-        int row = -1;
-        float rs = 0.f;
-        if (pos < tok_end) {
-          const int idx = p.indices[(size_t)b * p.topk + pos];
-          if (idx >= 0) {
-            row = p.page_size ? p.page_table[(size_t)b * p.pages_per_seq + idx / p.page_size] * p.page_size +
-                                    idx % p.page_size
-                              : idx;
-            if (kFp8) rs = p.kv_row_scale[row];
-          }
-        }
-        s_row[slot * kTile + ptid] = row;
-        if (kFp8) s_rsc[slot * kTile + ptid] = rs;
-      }
-      named_bar_sync(1, kProd);
+      const int slot = t & 1, rs = t % kRing;
+      if (!mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1)) break;
       const uint32_t tbase = sbase + kSmemKV + slot * kTileBytes;
       if constexpr (!kFp8) {
-        // 64 rows x 72 chunks of 16 B; consecutive lanes take consecutive
-        // chunks of a row (coalesced); padding rows are zero-filled.
-        for (int c = ptid; c < kTile * 72; c += kProd) {
-          const int tok = c / 72, ch = c - tok * 72;
-          const int row = s_row[slot * kTile + tok];
-          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16 + ch * 16;
-          cp_async_16(tbase + (ch >> 3) * kAtomBytes + sw128_off(tok, ch & 7), src, row >= 0 ? 16u : 0u);
+        // Loader warp w copies atoms w, w+4, w+8: 64 rows x 8 chunks of 16 B
+        // per atom, 16 per lane; each warp instruction covers four whole
+        // 128-byte row segments (coalesced).  Padding rows are zero-filled
+        // (source size 0).  The atom's barrier receives this warp's 32
+        // asynchronous arrivals.
+        const int lw = lt >> 5;
+        int rows[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) rows[u] = s_row[rs * 64 + 4 * u + (lane >> 3)];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
+        if (t >= 2 && !mbar_wait(BAR(BAR_KVE + slot), ((t >> 1) - 1) & 1)) break;
+        if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
+        const int j = lane & 7;
+#pragma unroll 1
+        for (int a = lw; a < kAtoms; a += 4) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int tok = 4 * u + (lane >> 3);
+            const int row = rows[u];
+            const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16 + a * 128 + j * 16;
+            cp_async_16(tbase + a * kAtomBytes + sw128_off(tok, j), src, row >= 0 ? 16u : 0u);
+          }
         }
-        cp_async_mbar_arrive_noinc(BAR(BAR_KVF + slot));
-        mbar_arrive(BAR(BAR_KVF + slot));
+        cp_async_mbar_arrive_noinc(BAR(BAR_KVF + slot * kAtoms));
+        if (lt == 0 && t == 2) SMLA_TRACE_EV(57);
       } else {
-        // 64 rows x 36 chunks of 16 fp8 codes; all loads issued first, then
-        // converted exactly to bf16 and stored swizzled.
-        constexpr int kPer = kTile * 36 / kProd;
-        static_assert(kTile * 36 % kProd == 0, "fp8 producer split");
-        uint4 v[kPer];
+        // thread (tok = lt/4, sub = lt%4): 16 codes of every atom; loads are
+        // issued before the stage is free and converted once it is
+        const int tok = lt >> 2, sub = lt & 3;
+        const int row = s_row[rs * 64 + tok];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
+        uint4 v[kAtoms];
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          const int c = ptid + u * kProd;
-          const int tok = c / 36, ch = c - tok * 36;
-          const int row = s_row[slot * kTile + tok];
-          v[u] = row >= 0 ? ld_global_nc_v4(p.kv + (size_t)row * kRowBytesFp8 + ch * 16) : make_uint4(0, 0, 0, 0);
-        }
+        for (int a = 0; a < kAtoms; ++a)
+          v[a] = row >= 0 ? ld_global_nc_v4(p.kv + (size_t)row * kRowBytesFp8 + a * 64 + sub * 16)
+                          : make_uint4(0, 0, 0, 0);
+        if (t >= 2 && !mbar_wait(BAR(BAR_KVE + slot), ((t >> 1) - 1) & 1)) break;
+        if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-          const int c = ptid + u * kProd;
-          const int tok = c / 36, ch = c - tok * 36;
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        for (int a = 0; a < kAtoms; ++a) {
           uint4 lo, hi;
-          lo.x = e4m3x2_to_bf16x2((uint16_t)(w[0] & 0xFFFF));
-          lo.y = e4m3x2_to_bf16x2((uint16_t)(w[0] >> 16));
-          lo.z = e4m3x2_to_bf16x2((uint16_t)(w[1] & 0xFFFF));
-          lo.w = e4m3x2_to_bf16x2((uint16_t)(w[1] >> 16));
-          hi.x = e4m3x2_to_bf16x2((uint16_t)(w[2] & 0xFFFF));
-          hi.y = e4m3x2_to_bf16x2((uint16_t)(w[2] >> 16));
-          hi.z = e4m3x2_to_bf16x2((uint16_t)(w[3] & 0xFFFF));
-          hi.w = e4m3x2_to_bf16x2((uint16_t)(w[3] >> 16));
-          // dims [16ch, 16ch+16) = bf16 chunks 2ch, 2ch+1 of the row
-          const int j0 = (ch & 3) * 2;
-          const uint32_t rb = tbase + (ch >> 2) * kAtomBytes;
-          st_shared_v4(rb + sw128_off(tok, j0), lo);
-          st_shared_v4(rb + sw128_off(tok, j0 + 1), hi);
+          lo.x = e4m3x2_to_bf16x2((uint16_t)(v[a].x & 0xFFFF));
+          lo.y = e4m3x2_to_bf16x2((uint16_t)(v[a].x >> 16));
+          lo.z = e4m3x2_to_bf16x2((uint16_t)(v[a].y & 0xFFFF));
+          lo.w = e4m3x2_to_bf16x2((uint16_t)(v[a].y >> 16));
+          hi.x = e4m3x2_to_bf16x2((uint16_t)(v[a].z & 0xFFFF));
+          hi.y = e4m3x2_to_bf16x2((uint16_t)(v[a].z >> 16));
+          hi.z = e4m3x2_to_bf16x2((uint16_t)(v[a].w & 0xFFFF));
+          hi.w = e4m3x2_to_bf16x2((uint16_t)(v[a].w >> 16));
+          const uint32_t rb = tbase + a * kAtomBytes;
+          st_shared_v4(rb + sw128_off(tok, 2 * sub), lo);
+          st_shared_v4(rb + sw128_off(tok, 2 * sub + 1), hi);
         }
+        // one proxy fence for the whole tile: generic stores -> tensor-core reads
         fence_proxy_async_smem();
-        mbar_arrive(BAR(BAR_KVF + slot));
+        if (lt == 0 && t == 2) SMLA_TRACE_EV(57);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(BAR_KVF + slot * kAtoms));
       }
     }
-    cp_async_wait_all();
-  } else if (warp == 4) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(BAR(BAR_Q), 0);
-      int ns = 0, npv = 0;
-      uint64_t t_last = globaltimer_ns();
-      while (ok && npv < ntiles) {
-        bool progressed = false;
-        if (ns < ntiles && ns <= npv + 1) {
-          const int slot = ns & 1;
-          if (mbar_test_wait(BAR(BAR_KVF + slot), (ns >> 1) & 1) &&
-              (ns < 2 || mbar_test_wait(BAR(BAR_SE + slot), ((ns >> 1) - 1) & 1))) {
-            fence_proxy_async_smem();
-            tc_fence_after();
-            const uint32_t qa = sbase + kSmemQ;
-            const uint32_t ka = sbase + kSmemKV + slot * kTileBytes;
-            const uint32_t d = tmem + kColS + 64u * (uint32_t)slot;
-#pragma unroll 4
-            for (int k = 0; k < kDqk / 16; ++k) {
-              const uint32_t off = (k >> 2) * kAtomBytes + (k & 3) * 32;
-              mma_bf16(d, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + off, 16, 1024), kIdescS,
-                       k > 0 ? 1u : 0u);
-            }
-            tc_commit(BAR(BAR_SF + slot));
-            ++ns;
-            progressed = true;
-          }
-        }
-        if (npv < ns && mbar_test_wait(BAR(BAR_PF), npv & 1)) {
+    if (!kFp8) cp_async_wait_all();
+  } else if (warp == kWarpS || warp == kWarpPV) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two warps issue tensor-core work, each blocking (in hardware) on one
+    // barrier at a time instead of polling: warp kWarpS computes S(t) as the
+    // atoms of tile t land; warp kWarpPV computes PV(t) once P(t) is written.
+    // Each warp runs with warp-uniform state and one elected lane issues.
+    // tcgen05.commit tracks the issuing thread's own MMAs.
+    bool ok = mbar_wait(BAR(BAR_Q), 0);
+    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
+    if (lane == 0 && warp == kWarpS) SMLA_TRACE_EV(2);
+    // Descriptors are built once; a K step or column block is a constant
+    // added to the start-address field (byte offset >> 4; the field does not
+    // overflow within the 227 KB window).
+    auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+      return __shfl_sync(0xffffffffu, (int)mbar_wait(bar, parity), 0) != 0;
+    };
+    if (warp == kWarpS) {
+      const uint64_t dq = sw128_desc(sbase + kSmemQ, 16, 1024);
+      const uint64_t dk0 = sw128_desc(sbase + kSmemKV, 16, 1024);
+      const uint64_t dk1 = sw128_desc(sbase + kSmemKV + kTileBytes, 16, 1024);
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int slot = t & 1;
+        // S(t) reuses the S buffer of S(t-2): its softmax must have read it
+        if (t >= 2) {
+          ok = wait_all(BAR(BAR_SE + slot), ((t >> 1) - 1) & 1);
+          if (!ok) break;
           tc_fence_after();
-          const int slot = npv & 1;
-          const uint32_t va = sbase + kSmemKV + slot * kTileBytes;
-          const uint32_t pa = sbase + kSmemP;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_bf16(tmem + kColO + 64u * (uint32_t)c,
-                       sw128_desc(va + (2 * c) * kAtomBytes + kk * 2048, kAtomBytes, 1024),
-                       sw128_desc(pa + kk * 32, 16, 1024), kIdescPV, (npv > 0 || kk > 0) ? 1u : 0u);
-            }
-          }
-          tc_commit(BAR(BAR_KVE + slot));
-          tc_commit(BAR(BAR_PVD));
-          ++npv;
-          progressed = true;
         }
-        if (progressed) {
-          t_last = globaltimer_ns();
-        } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
-          atomicOr(&g_error_word, 1u);
-          ok = false;
+        const uint64_t dk = slot ? dk1 : dk0;
+        const uint32_t d = tmem + kColS + 64u * (uint32_t)slot;
+        ok = wait_all(BAR(BAR_KVF + slot * kAtoms), (t >> 1) & 1);
+        if (!ok) break;
+        if (lane == 0 && t < 8) SMLA_TRACE_EV(24 + t);
+        // 36 K steps: atom a (+512 in the descriptor), 16-element step kk (+2)
+        mma_set_elect(d, dq, dk, kIdescS);
+#pragma unroll
+        for (int k = 1; k < kDqk / 16; ++k) {
+          const uint64_t off = (uint64_t)((k >> 2) * (kAtomBytes >> 4) + (k & 3) * 2);
+          mma_acc_elect(d, dq + off, dk + off, kIdescS);
         }
+        if (!ok) break;
+        commit_elect(BAR(BAR_SF + slot));
+        if (lane == 0 && t < 8) SMLA_TRACE_EV(8 + t);
       }
-      // drain: every MMA this thread issued has completed before teardown
-      tc_commit(BAR(BAR_FIN));
-      mbar_wait(BAR(BAR_FIN), 0);
+    } else {
+      const uint64_t dv0 = sw128_desc(sbase + kSmemKV, kAtomBytes, 1024);
+      const uint64_t dv1 = sw128_desc(sbase + kSmemKV + kTileBytes, kAtomBytes, 1024);
+      const uint64_t dp = sw128_desc(sbase + kSmemP, 16, 1024);
+      for (int t = 0; ok && t < ntiles; ++t) {
+        ok = wait_all(BAR(BAR_PF), t & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const int slot = t & 1;
+        const uint64_t dv = slot ? dv1 : dv0;
+        // chunk c: dims 128c.. = atoms 2c, 2c+1 (A, MN-major); K step kk:
+        // tokens 16kk.. = +2048 B in A, +32 B in P
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t d = tmem + kColO + 64u * (uint32_t)c;
+          const uint64_t a0 = dv + (uint64_t)(c * (2 * kAtomBytes >> 4));
+          if (t == 0) mma_set_elect(d, a0, dp, kIdescPV);
+          else mma_acc_elect(d, a0, dp, kIdescPV);
+          mma_acc_elect(d, a0 + 128, dp + 2, kIdescPV);
+          mma_acc_elect(d, a0 + 256, dp + 4, kIdescPV);
+          mma_acc_elect(d, a0 + 384, dp + 6, kIdescPV);
+        }
+        commit_elect(BAR(BAR_KVE + slot));
+        commit_elect(BAR(BAR_PVD));
+        if (lane == 0 && t < 8) SMLA_TRACE_EV(16 + t);
+      }
     }
+    // drain: every MMA this warp issued has completed before teardown
+    // (each warp has its own completion barrier)
+    commit_elect(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2));
+    mbar_wait(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2), 0);
   } else {
     // ------------------------------------------------------------ softmax
     const int h = 16 * warp + (lane & 15);   // head row of this thread
@@ -544,21 +686,30 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f, l_pv = 0.f;
     bool aborted = false;
     for (int i = 0; i < ntiles; ++i) {
-      const int sb = i & 1;
-      // S(i) is in TMEM; the load barrier of the tile is complete too (S
-      // consumed it), and waiting on it here acquires the producers' row
-      // table and row scales for this tile.
-      const bool f1 = !mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_KVF + sb), (i >> 1) & 1);
+      const int sb = i & 1, rs = i % kRing;
+      const bool f1 = !mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_IXF + rs), (i / kRing) & 1);
       if (group_any(f1, 2, 128)) { aborted = true; break; }
       tc_fence_after();
       float s[32];
       tmem_ld_16x32bx2_x32(tmem + lane_base + kColS + 64u * (uint32_t)sb, s);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(BAR(BAR_SE + sb));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_SE + sb));
 
-      const int* rows = s_row + sb * kTile + half * 32;
-      const float* rsc = s_rsc + sb * kTile + half * 32;
+      int rows[32];
+      float rsc[32];
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const int4 r4 = *reinterpret_cast<const int4*>(s_row + rs * 64 + half * 32 + j);
+        rows[j] = r4.x; rows[j + 1] = r4.y; rows[j + 2] = r4.z; rows[j + 3] = r4.w;
+        if (kFp8) {
+          const float4 c4 = *reinterpret_cast<const float4*>(s_rsc + rs * 64 + half * 32 + j);
+          rsc[j] = c4.x; rsc[j + 1] = c4.y; rsc[j + 2] = c4.z; rsc[j + 3] = c4.w;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
       float tmax = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -578,13 +729,12 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       for (int j = 0; j < 32; j += 2) {
         const float p0 = s[j] == -INFINITY ? 0.f : ex2(s[j] - m_use);
         const float p1 = s[j + 1] == -INFINITY ? 0.f : ex2(s[j + 1] - m_use);
+        lsum += p0 + p1;
         if constexpr (kFp8) {
           pk[j / 2] = pack_bf16x2(p0 * rsc[j], p1 * rsc[j + 1]);
-          lsum += p0 + p1;
         } else {
           const uint32_t w = pack_bf16x2(p0, p1);
           pk[j / 2] = w;
-          lsum += p0 + p1;
           lsum_pv += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
         }
       }
@@ -621,7 +771,9 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(BAR(BAR_PF));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_PF));
+      if (threadIdx.x == 0 && i < 8) SMLA_TRACE_EV(32 + i);
     }
     // ---------------------------------------------------------- epilogue
     if (!aborted && ntiles > 0) {
@@ -629,7 +781,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       aborted = group_any(f, 2, 128);
       tc_fence_after();
     }
+    if (threadIdx.x == 0) SMLA_TRACE_EV(3);
     if (!aborted) {
+      float* s_invl = reinterpret_cast<float*>(smem + kEpiInvl);
+      float* s_lse = reinterpret_cast<float*>(smem + kEpiLse);
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       const bool any = l_tot > 0.f;
@@ -654,36 +809,54 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         }
         const int dim = (c >> 1) * 128 + 32 * warp + lane;
         const int h0 = (c & 1) * 32;
+        float il[32];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float val = o[k] * s_invl[h0 + k];
-          if (direct) st_bf[(h0 + k) * kDv + dim] = __float2bfloat16_rn(val);
-          else st_f[(h0 + k) * kDv + dim] = val;
+        for (int k = 0; k < 32; k += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(s_invl + h0 + k);
+          il[k] = v4.x; il[k + 1] = v4.y; il[k + 2] = v4.z; il[k + 3] = v4.w;
+        }
+        if (direct) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) st_bf[(h0 + k) * kDv + dim] = __float2bfloat16_rn(o[k] * il[k]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) st_f[(h0 + k) * kDv + dim] = o[k] * il[k];
         }
       }
+      fence_proxy_async_smem();
       named_bar_sync(2, 128);
-      const int tid = threadIdx.x;  // 0..127
-      if (direct) {
-        const uint4* src = reinterpret_cast<const uint4*>(st_bf);
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)b * kH * kDv);
-        for (int i = tid; i < kH * kDv * 2 / 16; i += 128) dst[i] = src[i];
-        if (half == 0) p.lse[(size_t)b * kH + h] = s_lse[h];
-      } else {
-        const size_t part = (size_t)b * p.nsplit + split;
-        const uint4* src = reinterpret_cast<const uint4*>(st_f);
-        uint4* dst = reinterpret_cast<uint4*>(p.part_o + part * kH * kDv);
-        for (int i = tid; i < kH * kDv * 4 / 16; i += 128) dst[i] = src[i];
-        if (half == 0) p.part_lse[part * kH + h] = s_lse[h];
+      if (threadIdx.x == 0) {
+        SMLA_TRACE_EV(4);
+        if (direct) {
+          uint8_t* dst = reinterpret_cast<uint8_t*>(p.out + (size_t)b * kH * kDv);
+          for (int k = 0; k < 2; ++k)
+            bulk_store_s2g(dst + k * 32768, sbase + kSmemKV + k * 32768, 32768u);
+        } else {
+          const size_t part = (size_t)b * p.nsplit + split;
+          uint8_t* dst = reinterpret_cast<uint8_t*>(p.part_o + part * kH * kDv);
+          for (int k = 0; k < 4; ++k)
+            bulk_store_s2g(dst + k * 32768, sbase + kSmemKV + k * 32768, 32768u);
+        }
+        bulk_commit();
+      }
+      if (half == 0) {
+        if (direct) p.lse[(size_t)b * kH + h] = s_lse[h];
+        else p.part_lse[((size_t)b * p.nsplit + split) * kH + h] = s_lse[h];
+      }
+      if (threadIdx.x == 0) {
+        bulk_wait_all();
+        SMLA_TRACE_EV(5);
       }
     }
     tc_fence_before();
   }
 
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kWarpS) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  SMLA_TRACE_EV(6);
 }
 
 // ============================================================ combine kernel
@@ -772,6 +945,37 @@ static size_t partial_bytes(int batch, int nsplit) {
   return ((o + l + 255) / 256) * 256;
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
+// point (no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  return fn;
+}
+// 2-D bf16 tensor [outer][inner] with rows `row_bytes` apart; box
+// box_inner x box_outer elements, 128-byte swizzle, zero fill out of range.
+static bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                           uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The shared-memory opt-in is set once per device (an idempotent call, so a
 // race between threads is harmless); later calls, including calls made
 // while a stream is being captured into a CUDA graph, skip it.
@@ -818,6 +1022,8 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
     if (workspace_bytes < partial_bytes(shape->batch, n)) return SMLA_ERR_WORKSPACE;
   }
   SplitParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (!encode_bf16_2d(&prm.tmap_q, q, kDqk, (uint64_t)shape->batch * kH, kRowBytesBf16, 64, 64)) return SMLA_ERR_CUDA;
   prm.q = static_cast<const uint8_t*>(q);
   prm.kv = static_cast<const uint8_t*>(kv_cache);
   prm.kv_row_scale = kv_row_scale;
@@ -926,3 +1132,16 @@ smla_status sparse_mla_get_device_error(uint32_t* code) {
 }
 
 }  // extern "C"
+
+#ifdef SMLA_TRACE
+// Development-only accessor of the timeline probe (not part of the ABI).
+extern "C" int smla_trace_read(unsigned long long* host, size_t n) {
+  if (n > sizeof(smla::g_trace) / sizeof(unsigned long long)) n = sizeof(smla::g_trace) / sizeof(unsigned long long);
+  if (cudaMemcpyFromSymbol(host, smla::g_trace, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
+  return (int)n;
+}
+extern "C" int smla_trace_clear(void) {
+  static unsigned long long zeros[256 * 64];
+  return cudaMemcpyToSymbol(smla::g_trace, zeros, sizeof(zeros)) == cudaSuccess ? 0 : -1;
+}
+#endif
