@@ -26,9 +26,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -53,52 +51,62 @@ def load_peaks():
 
 
 # --------------------------------------------------------------- clocks
+_REASON_BITS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
+
+
+def _nvml_sampler(conn, busid: str, period_s: float):
+    """Runs in a spawned process: samples the SM clock and the clock event
+    reasons of one GPU through NVML until told to stop."""
+    import time as _t
+    import pynvml
+    pynvml.nvmlInit()
+    h = pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+    reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+        pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+    maxsm = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    samples = []
+    conn.send("ready")
+    while not conn.poll(0):
+        samples.append((_t.time(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(reasons(h))))
+        _t.sleep(period_s)
+    conn.recv()
+    conn.send((maxsm, samples))
+
+
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples clocks in a separate process (no GIL contention with the timed
+    loop); summary() keeps the samples taken inside [t0, t1]."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, device):
         self.proc = None
-        self.file = None
-
-    def __enter__(self):
+        self.conn = None
         try:
-            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
-        except Exception:
+            import multiprocessing as mp
+            pr = torch.cuda.get_device_properties(device)
+            busid = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            ctx = mp.get_context("spawn")
+            self.conn, child = ctx.Pipe()
+            self.proc = ctx.Process(target=_nvml_sampler, args=(child, busid, 0.001), daemon=True)
+            self.proc.start()
+            if not self.conn.poll(60) or self.conn.recv() != "ready":
+                raise RuntimeError("sampler did not start")
+        except Exception as e:  # no NVML: report clocks as unavailable
+            self.error = str(e)
             self.proc = None
-        return self
 
-    def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-
-    def summary(self):
-        if self.proc is None or self.file is None:
-            return None
-        self.file.flush()
-        rows = []
-        for line in open(self.file.name):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
-        os.unlink(self.file.name)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+    def summary(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML sampler unavailable: " + getattr(self, "error", "")}
+        self.conn.send("stop")
+        maxsm, samples = self.conn.recv()
+        self.proc.join(timeout=10)
+        inside = [x for x in samples if t0 <= x[0] <= t1]
+        if not inside:  # the region was shorter than one sample: take the nearest
+            inside = sorted(samples, key=lambda x: min(abs(x[0] - t0), abs(x[0] - t1)))[:1]
+        reasons = sorted({name for _, _, r in inside for bit, name in _REASON_BITS.items() if r & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in inside) if inside else None, "sm_max_mhz": maxsm,
+                "reasons": reasons, "samples": len(inside)}
 
 
 # --------------------------------------------------------------- helpers
@@ -113,36 +121,27 @@ def roofline_us(w, peak_gbs, peak_tflops):
 
 
 class Runner:
-    """Preallocated outputs/workspace for one workload on one device."""
+    """One workload on one device with a pre-marshalled decode call."""
 
     def __init__(self, w, dev):
         from sparse_mla_decode_05_b200 import api
         self.api = api
         self.w = w
         self.t = to_dev(w, dev)
-        self.shape = api.shape_for(self.t["q"], self.t["kv"], self.t["indices"], page_table=self.t["page_table"],
-                                   page_size=w.page_size)
-        self.nsplit = api.plan_nsplit(self.shape)
-        ws = api.workspace_size(self.shape)
-        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
-        self.out = torch.empty((w.batch, 64, 512), dtype=torch.bfloat16, device=dev)
-        self.lse = torch.empty((w.batch, 64), dtype=torch.float32, device=dev)
-
-    def decode(self, q=None, indices=None):
         t = self.t
-        return self.api.decode(t["q"] if q is None else q, t["kv"], t["indices"] if indices is None else indices,
-                               self.w.scale, kv_row_scale=t["kv_row_scale"], page_table=t["page_table"],
-                               page_size=self.w.page_size, out=self.out, lse=self.lse, workspace=self.ws)
+        self.plan = api.DecodePlan(t["q"], t["kv"], t["indices"], w.scale, kv_row_scale=t["kv_row_scale"],
+                                   page_table=t["page_table"], page_size=w.page_size)
+        self.nsplit = self.plan.nsplit
+        self.out, self.lse = self.plan.out, self.plan.lse
+
+    def decode(self):
+        self.plan.run()
 
     def split_only(self):
-        t = self.t
-        return self.api.decode_split(t["q"], t["kv"], t["indices"], self.w.scale, kv_row_scale=t["kv_row_scale"],
-                                     page_table=t["page_table"], page_size=self.w.page_size, out=self.out,
-                                     lse=self.lse, workspace=self.ws)
+        self.plan.run_split()
 
     def combine_only(self):
-        po, pl = self.api.partial_views(self.ws, self.w.batch, self.nsplit)
-        return self.api.combine(po, pl, out=self.out, lse=self.lse)
+        self.plan.run_combine()
 
     @property
     def launches_per_step(self):
@@ -216,7 +215,7 @@ def oracle_time(w: inputs.Workload, budget_s: float = 15.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--workload", default=HEADLINE, choices=list(inputs.CONFIG_NAMES))
@@ -276,13 +275,15 @@ def main():
         torch.cuda.synchronize()
 
     # --- headline: device-resident inputs, whole call
+    clk = ClockSampler(dev)
     barrier()
-    with ClockSampler(local) as clk:
-        t_wall0 = time.perf_counter()
-        times = time_device(r.decode, args.steps, args.warmup, flush, stream)
-        barrier()
-        t_wall = time.perf_counter() - t_wall0
-    clocks = clk.summary()
+    t_wall0 = time.perf_counter()
+    t_clk0 = time.time()
+    times = time_device(r.decode, args.steps, args.warmup, flush, stream)
+    barrier()
+    t_clk1 = time.time()
+    t_wall = time.perf_counter() - t_wall0
+    clocks = clk.summary(t_clk0, t_clk1)
     ms = float(np.mean(times))
     if world > 1:
         import torch.distributed as dist
@@ -312,6 +313,8 @@ def main():
     hlse = torch.empty(r.lse.shape, dtype=r.lse.dtype).pin_memory()
     dq = torch.empty_like(r.t["q"])
     didx = torch.empty_like(r.t["indices"])
+    e2e_plan = api.DecodePlan(dq, r.t["kv"], didx, w.scale, kv_row_scale=r.t["kv_row_scale"],
+                              page_table=r.t["page_table"], page_size=w.page_size)
     h2d = hq.numel() * 2 + hidx.numel() * 4 + (0 if hpt is None else hpt.numel() * 4)
     d2h = hout.numel() * 2 + hlse.numel() * 4
 
@@ -320,9 +323,9 @@ def main():
         didx.copy_(hidx, non_blocking=True)
         if hpt is not None:
             r.t["page_table"].copy_(hpt, non_blocking=True)
-        r.decode(q=dq, indices=didx)
-        hout.copy_(r.out, non_blocking=True)
-        hlse.copy_(r.lse, non_blocking=True)
+        e2e_plan.run()
+        hout.copy_(e2e_plan.out, non_blocking=True)
+        hlse.copy_(e2e_plan.lse, non_blocking=True)
 
     e2e_times = time_device(e2e_step, max(10, args.steps // 2), 3, flush, stream)
     e2e_ms = float(np.mean(e2e_times))

@@ -189,3 +189,55 @@ def device_error() -> int:
     if st not in (0, 5):
         raise SmlaError(st, "sparse_mla_get_device_error")
     return code.value
+
+
+class DecodePlan:
+    """A decode call with its arguments marshalled once.
+
+    For repeated calls on fixed buffers (serving loops, CUDA-graph capture,
+    benchmarking): run() is a single call into the library with no
+    per-call Python-side checks.  The tensors must stay alive and keep their
+    addresses while the plan is in use.
+    """
+
+    def __init__(self, q, kv, indices, scale: float, *, kv_row_scale=None, page_table=None,
+                 page_size: int = 0, nsplit: int = 0, out=None, lse=None, workspace=None):
+        _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size)
+        self.shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
+        dev = q.device
+        self.nsplit = plan_nsplit(self.shape)
+        self.out = out if out is not None else torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
+        self.lse = lse if lse is not None else torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
+        ws = workspace_size(self.shape)
+        self.workspace = workspace if workspace is not None or ws == 0 else \
+            torch.empty(ws, dtype=torch.uint8, device=dev)
+        self._keep = (q, kv, indices, kv_row_scale, page_table)
+        wsp = _ptr(self.workspace)
+        wsn = 0 if self.workspace is None else self.workspace.numel()
+        self._stream = _stream(dev)
+        self._args = (ctypes.byref(self.shape), _ptr(q), _ptr(kv), _ptr(kv_row_scale), _ptr(page_table),
+                      _ptr(indices), float(scale), _ptr(self.out), _ptr(self.lse), wsp, wsn)
+        self._split_args = self._args + (None,)
+        if self.nsplit > 1:
+            po, pl = partial_views(self.workspace, q.shape[0], self.nsplit)
+            self._combine_args = (q.shape[0], H, D_V, self.nsplit, _ptr(po), _ptr(pl), _ptr(self.out),
+                                  _ptr(self.lse))
+        else:
+            self._combine_args = None
+
+    def run(self, stream=None):
+        st = lib.sparse_mla_decode(*self._args, self._stream if stream is None else stream)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_decode")
+
+    def run_split(self, stream=None):
+        st = lib.sparse_mla_decode_split(*self._split_args, self._stream if stream is None else stream)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_decode_split")
+
+    def run_combine(self, stream=None):
+        if self._combine_args is None:
+            return
+        st = lib.sparse_mla_combine(*self._combine_args, self._stream if stream is None else stream)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_combine")

@@ -42,7 +42,6 @@
 // records an error bit in a device word, drains its own copies and MMAs,
 // frees TMEM and exits.
 
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -66,41 +65,44 @@ constexpr int kRowBytesBf16 = kDqk * 2;             // 1152
 constexpr int kRowBytesFp8 = kDqk;                  // 576
 
 // shared memory map (offsets from the 1024-aligned dynamic shared base)
-constexpr int kSmemQ = 0;                           // Q   [9 atoms][64 heads][128 B]
-constexpr int kSmemKV = kSmemQ + kTileBytes;        // KV  [2 stages][9 atoms][64 tok][128 B]
-constexpr int kSmemP = kSmemKV + 2 * kTileBytes;    // P   [64 heads][64 tok] bf16 (K-major)
+constexpr int kStages = 3;                          // KV tile stages
+constexpr int kSmemKV = 0;                          // KV  [3 stages][9 atoms][64 tok][128 B]
+constexpr int kSmemP = kSmemKV + kStages * kTileBytes;  // P [64 heads][64 tok] bf16 (K-major)
 constexpr int kSmemAux = kSmemP + 64 * 128;
 constexpr int kRing = 4;                            // resolved-row ring depth (tiles)
 // barrier indices
-constexpr int BAR_Q = 0;
-constexpr int BAR_KVF = 1;                          // [2 stages][9 atoms]
-constexpr int BAR_KVE = BAR_KVF + 2 * kAtoms;       // [2]
-constexpr int BAR_SF = BAR_KVE + 2;                 // [2]
-constexpr int BAR_SE = BAR_SF + 2;                  // [2]
-constexpr int BAR_PF = BAR_SE + 2;
-constexpr int BAR_PVD = BAR_PF + 1;
-constexpr int BAR_FIN = BAR_PVD + 1;
-constexpr int BAR_FIN2 = BAR_FIN + 1;
-constexpr int BAR_IXF = BAR_FIN2 + 1;               // [kRing]
-constexpr int BAR_IXE = BAR_IXF + kRing;            // [kRing]
+constexpr int BAR_KVF = 0;                          // [kStages] tile landed
+constexpr int BAR_KVE = BAR_KVF + kStages;          // [kStages] tile consumed (PV done)
+constexpr int BAR_SF = BAR_KVE + kStages;           // [2] S(t) in TMEM
+constexpr int BAR_SE = BAR_SF + 2;                  // [2] S(t) read by the softmax
+constexpr int BAR_PF = BAR_SE + 2;                  // P(t) written
+constexpr int BAR_PVD = BAR_PF + 1;                 // PV(t) done
+constexpr int BAR_FIN = BAR_PVD + 1;                // drain, S issuer
+constexpr int BAR_FIN2 = BAR_FIN + 1;               // drain, PV issuer
+constexpr int BAR_QT = BAR_FIN2 + 1;                // query written to TMEM
+constexpr int BAR_QS = BAR_QT + 1;                  // query staged in shared memory
+constexpr int BAR_IXF = BAR_QS + 1;                 // [kRing] rows resolved
+constexpr int BAR_IXE = BAR_IXF + kRing;            // [kRing] rows consumed
 constexpr int kNumBars = BAR_IXE + kRing;
 constexpr int kAuxBars = kSmemAux;
 constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
 constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
 constexpr int kAuxRsc = kAuxRow + kRing * 64 * 4;   // f32  [kRing][64] fp8 row scales
-constexpr int kAuxAlpha = kAuxRsc + kRing * 64 * 4; // f32  [64] rescale factors
-constexpr int kAuxEnd = kAuxAlpha + 64 * 4;
+constexpr int kAuxEnd = kAuxRsc + kRing * 64 * 4;
 constexpr int kSmemBytes = kAuxEnd;
-// epilogue scratch inside the (then idle) P buffer
-constexpr int kEpiInvl = kSmemP;                    // f32 [64] 1/l
-constexpr int kEpiLse = kSmemP + 256;               // f32 [64] lse
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
-static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxAlpha % 16 == 0, "aux arrays are read as 16-byte vectors");
+static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0, "aux arrays are read as 16-byte vectors");
 
-// TMEM columns (512 allocated): O^T chunks at 0..255, S buffers at 256 and 320
+// Tensor memory (512 columns x 128 lanes).  Each warp quarter (32 lanes)
+// holds 16 heads; an M=64 operand or accumulator uses lanes 0-15 or 16-31
+// of every quarter.
+//   lanes 0-15 : Q (A operand of S, bf16 packed two per column) cols [0,288)
+//                S buffers (fp32)                          cols [288,416)
+//   lanes 16-31: O (fp32, 64 heads x 512 dims)             cols [0,512)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0;
-constexpr uint32_t kColS = 256;
+constexpr uint32_t kColQ = 0;
+constexpr uint32_t kColS = 288;
+constexpr uint32_t kLaneO = 16;
 
 // Lazy rescaling: keep the running max until a new max exceeds it by more
 // than 2^8 (probabilities stay <= 256; results are unchanged).
@@ -112,16 +114,17 @@ constexpr uint32_t make_idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
-constexpr uint32_t kIdescS = make_idesc(64, 64, false, false);    // S  = Q K^T
-constexpr uint32_t kIdescPV = make_idesc(128, 64, true, false);   // O^T = V^T P^T
+constexpr uint32_t kIdescS = make_idesc(64, 64, false, false);    // S = Q K^T   (Q from TMEM)
+constexpr uint32_t kIdescPV = make_idesc(64, 256, false, true);   // O += P V    (V MN-major)
 
 // Bounded waits give up after this many SM clock cycles (about 2 s).
 constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // warps 0-3 softmax/epilogue, 4 S-MMA issuer (+ TMEM allocator), 5 PV-MMA
-// issuer, 6 index resolver, 7.. loaders (bf16 rows: four warps issuing
-// 16-byte cp.async; fp8 rows: eight warps that load, convert and store)
-constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kWarpLoad0 = 7;
+// issuer, 6-9 index resolvers (warp 6+k owns the tiles t = k mod 4), 10..
+// loaders (bf16 rows: four warps issuing 16-byte cp.async; fp8 rows: eight
+// warps that load, convert and store)
+constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kIdxWarps = 4, kWarpLoad0 = kWarpIdx + kIdxWarps;
 template <bool kFp8>
 struct Cfg {
   static constexpr int kLoadWarps = kFp8 ? 8 : 4;
@@ -130,7 +133,6 @@ struct Cfg {
 };
 
 struct SplitParams {
-  CUtensorMap tmap_q;          // q as [B*64, 576]: box 64 x 64, 128B swizzle
   const uint8_t* q;            // [B, 64, 576] bf16
   const uint8_t* kv;           // rows of 1152 B (bf16) or 576 B (fp8 codes)
   const float* kv_row_scale;   // [N] (fp8)
@@ -276,10 +278,6 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
 // Warp-uniform MMA issue: the whole warp computes the (uniform) operands and
 // one elected lane executes the instruction.  D[tmem] = A . B ("set", first K
 // step) or D[tmem] += A . B ("acc").
@@ -299,6 +297,25 @@ __device__ __forceinline__ void mma_acc_elect(uint32_t d_tmem, uint64_t a_desc, 
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
+// Same with the A operand read from tensor memory (K-major): D = A[tmem] . B
+__device__ __forceinline__ void mma_ts_set_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.u32 p, 0, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_acc_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.eq.u32 p, 0, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc)
       : "memory");
 }
 __device__ __forceinline__ void commit_elect(uint32_t bar) {
@@ -328,13 +345,14 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x32(uint32_t taddr, float (&v)[
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-// 32 lanes x 32 bits x 32 columns: thread t reads lane base+t, columns [c, c+32)
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
+// 16 lanes x 32 columns, twice: threads 0-15 access columns [c, c+32) of
+// lanes base+0..15, threads 16-31 columns [c+256, c+288) of the same lanes.
+__device__ __forceinline__ void tmem_ld_16x32bx2_x32_h256(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 256;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
         "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
@@ -344,9 +362,9 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float (&v)[32]) {
+__device__ __forceinline__ void tmem_st_16x32bx2_x32_h256(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 256, "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
@@ -360,6 +378,17 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float (
       "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+// 16 lanes x 16 columns, twice: threads 0-15 write columns [c, c+16) of
+// lanes base+0..15, threads 16-31 columns [c+144, c+160) (the query's second
+// 288 dims).
+__device__ __forceinline__ void tmem_st_16x32bx2_x16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 144, "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 
@@ -401,12 +430,10 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
-      : "memory");
+__device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sdst),
+               "l"(gsrc), "r"(bytes), "r"(bar)
+               : "memory");
 }
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
@@ -441,28 +468,27 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 
   int* s_row = reinterpret_cast<int*>(smem + kAuxRow);
   float* s_rsc = reinterpret_cast<float*>(smem + kAuxRsc);
-  float* s_alpha = reinterpret_cast<float*>(smem + kAuxAlpha);
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(BAR_Q), 1);
-    for (int s = 0; s < 2; ++s) {
-      // tile barrier (the first of the stage's atom slots is used): bf16 ->
-      // every loader thread's asynchronous arrival; fp8 -> one per loader warp
-      mbar_init(BAR(BAR_KVF + s * kAtoms), kFp8 ? kLoad / 32 : kLoad);
+    // Arrivals are per warp (the warp synchronises, one lane arrives), except
+    // where a copy engine arrives: mbarrier arrivals are serialised.
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(BAR(BAR_KVF + s), kFp8 ? kLoad / 32 : kLoad);  // fp8: loader warps; bf16: async copies
       mbar_init(BAR(BAR_KVE + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(BAR_SF + s), 1);
-      mbar_init(BAR(BAR_SE + s), 4);      // one arrival per softmax warp
+      mbar_init(BAR(BAR_SE + s), 4);
     }
     mbar_init(BAR(BAR_PF), 4);
     mbar_init(BAR(BAR_PVD), 1);
     mbar_init(BAR(BAR_FIN), 1);
     mbar_init(BAR(BAR_FIN2), 1);
-    // Arrivals are per warp (a warp synchronises, then one lane arrives):
-    // mbarrier arrivals are serialised, so hundreds of per-thread arrivals
-    // per tile would sit on the critical path.
+    mbar_init(BAR(BAR_QT), 4);
+    mbar_init(BAR(BAR_QS), 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(BAR(BAR_IXF + r), 1);
-      mbar_init(BAR(BAR_IXE + r), kLoad / 32 + 4);  // loader warps + softmax warps
+      mbar_init(BAR(BAR_IXE + r), kLoad / 32 + 4);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -476,11 +502,12 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kAuxTmem);
   SMLA_TRACE_EV(1);
 
-  if (warp == kWarpIdx) {
-    // ------------------------------------------------------------ index warp
-    // Resolves each tile's 64 entries to physical rows (and fp8 row scales)
-    // into a kRing-deep ring, running ahead of the loaders.  Loads are
-    // software-pipelined: index of tile t+2, page entry of t+1, scale of t.
+  if (warp >= kWarpIdx && warp < kWarpIdx + kIdxWarps) {
+    // ------------------------------------------------------------ index warps
+    // Resolve each tile's 64 entries to physical rows (and fp8 row scales)
+    // into the kRing-deep ring ahead of the loaders, and pull the rows into
+    // L2.  Warp k handles tiles t = k, k+4, ... (ring slot k), so four tiles'
+    // lookups are in flight at once.
     auto idx_at = [&](int t, int j) -> int {
       const int pos = tok_begin + t * kTile + j;
       return (t < ntiles && pos < tok_end) ? __ldg(p.indices + (size_t)b * p.topk + pos) : -1;
@@ -491,63 +518,79 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       return __ldg(p.page_table + (size_t)b * p.pages_per_seq + idx / p.page_size) * p.page_size +
              idx % p.page_size;
     };
-    int ia0 = idx_at(0, lane), ia1 = idx_at(0, lane + 32);
-    int ib0 = idx_at(1, lane), ib1 = idx_at(1, lane + 32);
-    int r0 = row_of(ia0), r1 = row_of(ia1);
-    for (int t = 0; t < ntiles; ++t) {
+    const int kw = warp - kWarpIdx;
+    // the 64 x 576 query (73,728 contiguous bytes) into the third KV stage,
+    // which no tile uses before the query has been moved to tensor memory
+    if (kw == 0 && lane == 0) {
+      mbar_arrive_expect_tx(BAR(BAR_QS), (uint32_t)kTileBytes);
+      bulk_load_g2s(sbase + kSmemKV + 2 * kTileBytes, p.q + (size_t)b * kH * kRowBytesBf16, (uint32_t)kTileBytes,
+                    BAR(BAR_QS));
+    }
+    // Software pipeline over this warp's tiles (step S = 4), every load
+    // consumed one iteration after it was issued: index of tile t+3S, page
+    // entry of t+2S, row scale of t+S (and the rows of t+S pulled into L2),
+    // then tile t is published.
+    constexpr uint32_t kRowBytes = kFp8 ? kRowBytesFp8 : kRowBytesBf16;
+    constexpr int S = kIdxWarps;
+    int i2_0 = idx_at(kw + 2 * S, lane), i2_1 = idx_at(kw + 2 * S, lane + 32);                 // tile t+2S
+    int r1_0 = row_of(idx_at(kw + S, lane)), r1_1 = row_of(idx_at(kw + S, lane + 32));         // tile t+S
+    int r0_0 = row_of(idx_at(kw, lane)), r0_1 = row_of(idx_at(kw, lane + 32));                 // tile t
+    float c0_0 = 0.f, c0_1 = 0.f;                                            // scale, tile t
+    if (kFp8) {
+      c0_0 = r0_0 >= 0 ? __ldg(p.kv_row_scale + r0_0) : 0.f;
+      c0_1 = r0_1 >= 0 ? __ldg(p.kv_row_scale + r0_1) : 0.f;
+    }
+    if (r0_0 >= 0) prefetch_l2(p.kv + (size_t)r0_0 * kRowBytes, kRowBytes);
+    if (r0_1 >= 0) prefetch_l2(p.kv + (size_t)r0_1 * kRowBytes, kRowBytes);
+    for (int t = kw; t < ntiles; t += S) {
       const int rs = t % kRing;
-      float c0 = 0.f, c1 = 0.f;
+      float c1_0 = 0.f, c1_1 = 0.f;
       if (kFp8) {
-        c0 = r0 >= 0 ? __ldg(p.kv_row_scale + r0) : 0.f;
-        c1 = r1 >= 0 ? __ldg(p.kv_row_scale + r1) : 0.f;
+        c1_0 = r1_0 >= 0 ? __ldg(p.kv_row_scale + r1_0) : 0.f;
+        c1_1 = r1_1 >= 0 ? __ldg(p.kv_row_scale + r1_1) : 0.f;
       }
-      const int n0 = row_of(ib0), n1 = row_of(ib1);
-      // rows of tile t+1 are known now: start pulling them into L2
-      {
-        constexpr uint32_t kRowBytes = kFp8 ? kRowBytesFp8 : kRowBytesBf16;
-        if (n0 >= 0) prefetch_l2(p.kv + (size_t)n0 * kRowBytes, kRowBytes);
-        if (n1 >= 0) prefetch_l2(p.kv + (size_t)n1 * kRowBytes, kRowBytes);
-      }
-      const int ic0 = idx_at(t + 2, lane), ic1 = idx_at(t + 2, lane + 32);
-      if (t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1)) break;
-      s_row[rs * 64 + lane] = r0;
-      s_row[rs * 64 + lane + 32] = r1;
+      if (r1_0 >= 0) prefetch_l2(p.kv + (size_t)r1_0 * kRowBytes, kRowBytes);
+      if (r1_1 >= 0) prefetch_l2(p.kv + (size_t)r1_1 * kRowBytes, kRowBytes);
+      const int r2_0 = row_of(i2_0), r2_1 = row_of(i2_1);
+      const int i3_0 = idx_at(t + 3 * S, lane), i3_1 = idx_at(t + 3 * S, lane + 32);
+      const bool fail = t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1);
+      if (__any_sync(0xffffffffu, fail)) break;  // warp-uniform exit
+      s_row[rs * 64 + lane] = r0_0;
+      s_row[rs * 64 + lane + 32] = r0_1;
       if (kFp8) {
-        s_rsc[rs * 64 + lane] = c0;
-        s_rsc[rs * 64 + lane + 32] = c1;
+        s_rsc[rs * 64 + lane] = c0_0;
+        s_rsc[rs * 64 + lane + 32] = c0_1;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXF + rs));
-      r0 = n0;
-      r1 = n1;
-      ib0 = ic0;
-      ib1 = ic1;
+      if (lane == 0 && t < 4) SMLA_TRACE_EV(58 + t);
+      r0_0 = r1_0; r0_1 = r1_1;
+      c0_0 = c1_0; c0_1 = c1_1;
+      r1_0 = r2_0; r1_1 = r2_1;
+      i2_0 = i3_0; i2_1 = i3_1;
     }
   } else if (warp >= kWarpLoad0) {
     // ------------------------------------------------------------ loaders
     const int lt = threadIdx.x - 32 * kWarpLoad0;  // 0 .. kLoad-1
-    if (lt == 0) {  // the 64 x 576 query: nine 64 x 64 TMA boxes, 128B-swizzled K-major
-      mbar_arrive_expect_tx(BAR(BAR_Q), (uint32_t)kTileBytes);
-      for (int a = 0; a < kAtoms; ++a)
-        tma_load_2d(sbase + kSmemQ + a * kAtomBytes, &p.tmap_q, a * 64, b * kH, BAR(BAR_Q));
-    }
     for (int t = 0; t < ntiles; ++t) {
-      const int slot = t & 1, rs = t % kRing;
-      if (!mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1)) break;
-      const uint32_t tbase = sbase + kSmemKV + slot * kTileBytes;
+      const int stage = t % kStages, rs = t % kRing;
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1))) break;  // warp-uniform
+      const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
       if constexpr (!kFp8) {
         // Loader warp w copies atoms w, w+4, w+8: 64 rows x 8 chunks of 16 B
         // per atom, 16 per lane; each warp instruction covers four whole
         // 128-byte row segments (coalesced).  Padding rows are zero-filled
-        // (source size 0).  The atom's barrier receives this warp's 32
-        // asynchronous arrivals.
+        // (source size 0).
         const int lw = lt >> 5;
         int rows[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) rows[u] = s_row[rs * 64 + 4 * u + (lane >> 3)];
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-        if (t >= 2 && !mbar_wait(BAR(BAR_KVE + slot), ((t >> 1) - 1) & 1)) break;
+        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+          break;
+        // stage 2 first holds the staged query
+        if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
         if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
         const int j = lane & 7;
 #pragma unroll 1
@@ -560,8 +603,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
             cp_async_16(tbase + a * kAtomBytes + sw128_off(tok, j), src, row >= 0 ? 16u : 0u);
           }
         }
-        cp_async_mbar_arrive_noinc(BAR(BAR_KVF + slot * kAtoms));
-        if (lt == 0 && t == 2) SMLA_TRACE_EV(57);
+        cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
       } else {
         // thread (tok = lt/4, sub = lt%4): 16 codes of every atom; loads are
         // issued before the stage is free and converted once it is
@@ -574,7 +616,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         for (int a = 0; a < kAtoms; ++a)
           v[a] = row >= 0 ? ld_global_nc_v4(p.kv + (size_t)row * kRowBytesFp8 + a * 64 + sub * 16)
                           : make_uint4(0, 0, 0, 0);
-        if (t >= 2 && !mbar_wait(BAR(BAR_KVE + slot), ((t >> 1) - 1) & 1)) break;
+        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+          break;
+        // stage 2 first holds the staged query
+        if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
         if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
 #pragma unroll
         for (int a = 0; a < kAtoms; ++a) {
@@ -593,92 +638,118 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         }
         // one proxy fence for the whole tile: generic stores -> tensor-core reads
         fence_proxy_async_smem();
-        if (lt == 0 && t == 2) SMLA_TRACE_EV(57);
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_KVF + slot * kAtoms));
+        if (lane == 0) mbar_arrive(BAR(BAR_KVF + stage));
       }
+      if (lt == 0 && t == 2) SMLA_TRACE_EV(57);
     }
     if (!kFp8) cp_async_wait_all();
   } else if (warp == kWarpS || warp == kWarpPV) {
     // ------------------------------------------------------------ MMA issuers
     // Two warps issue tensor-core work, each blocking (in hardware) on one
-    // barrier at a time instead of polling: warp kWarpS computes S(t) as the
-    // atoms of tile t land; warp kWarpPV computes PV(t) once P(t) is written.
-    // Each warp runs with warp-uniform state and one elected lane issues.
-    // tcgen05.commit tracks the issuing thread's own MMAs.
-    bool ok = mbar_wait(BAR(BAR_Q), 0);
-    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-    if (lane == 0 && warp == kWarpS) SMLA_TRACE_EV(2);
-    // Descriptors are built once; a K step or column block is a constant
-    // added to the start-address field (byte offset >> 4; the field does not
-    // overflow within the 227 KB window).
+    // barrier at a time: warp kWarpS computes S(t) once tile t has landed;
+    // warp kWarpPV computes PV(t) once P(t) is written.  Each warp runs with
+    // warp-uniform state and one elected lane issues; tcgen05.commit tracks
+    // the issuing thread's own MMAs.  Operand addresses advance by constants
+    // (shared descriptors: byte offset >> 4; tensor memory: columns).
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __shfl_sync(0xffffffffu, (int)mbar_wait(bar, parity), 0) != 0;
     };
+    bool ok = true;
     if (warp == kWarpS) {
-      const uint64_t dq = sw128_desc(sbase + kSmemQ, 16, 1024);
-      const uint64_t dk0 = sw128_desc(sbase + kSmemKV, 16, 1024);
-      const uint64_t dk1 = sw128_desc(sbase + kSmemKV + kTileBytes, 16, 1024);
+      uint64_t dk[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) dk[s] = sw128_desc(sbase + kSmemKV + s * kTileBytes, 16, 1024);
+      ok = wait_all(BAR(BAR_QT), 0);
+      tc_fence_after();
+      if (lane == 0) SMLA_TRACE_EV(2);
       for (int t = 0; ok && t < ntiles; ++t) {
-        const int slot = t & 1;
+        const int stage = t % kStages, sb = t & 1;
         // S(t) reuses the S buffer of S(t-2): its softmax must have read it
         if (t >= 2) {
-          ok = wait_all(BAR(BAR_SE + slot), ((t >> 1) - 1) & 1);
+          ok = wait_all(BAR(BAR_SE + sb), ((t >> 1) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
         }
-        const uint64_t dk = slot ? dk1 : dk0;
-        const uint32_t d = tmem + kColS + 64u * (uint32_t)slot;
-        ok = wait_all(BAR(BAR_KVF + slot * kAtoms), (t >> 1) & 1);
+        ok = wait_all(BAR(BAR_KVF + stage), (t / kStages) & 1);
         if (!ok) break;
         if (lane == 0 && t < 8) SMLA_TRACE_EV(24 + t);
-        // 36 K steps: atom a (+512 in the descriptor), 16-element step kk (+2)
-        mma_set_elect(d, dq, dk, kIdescS);
+        const uint64_t bk = stage == 0 ? dk[0] : (stage == 1 ? dk[1] : dk[2]);
+        const uint32_t d = tmem + kColS + 64u * (uint32_t)sb;
+        // 36 K steps: Q columns +8 per step (16 bf16); K descriptor: atom
+        // +512, 16-element step +2
+        mma_ts_set_elect(d, tmem + kColQ, bk, kIdescS);
 #pragma unroll
         for (int k = 1; k < kDqk / 16; ++k) {
           const uint64_t off = (uint64_t)((k >> 2) * (kAtomBytes >> 4) + (k & 3) * 2);
-          mma_acc_elect(d, dq + off, dk + off, kIdescS);
+          mma_ts_acc_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + off, kIdescS);
         }
-        if (!ok) break;
-        commit_elect(BAR(BAR_SF + slot));
+        commit_elect(BAR(BAR_SF + sb));
         if (lane == 0 && t < 8) SMLA_TRACE_EV(8 + t);
       }
     } else {
-      const uint64_t dv0 = sw128_desc(sbase + kSmemKV, kAtomBytes, 1024);
-      const uint64_t dv1 = sw128_desc(sbase + kSmemKV + kTileBytes, kAtomBytes, 1024);
+      uint64_t dv[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) dv[s] = sw128_desc(sbase + kSmemKV + s * kTileBytes, kAtomBytes, 1024);
       const uint64_t dp = sw128_desc(sbase + kSmemP, 16, 1024);
+      const uint32_t o0 = tmem + (kLaneO << 16);
       for (int t = 0; ok && t < ntiles; ++t) {
         ok = wait_all(BAR(BAR_PF), t & 1);
         if (!ok) break;
         tc_fence_after();
-        const int slot = t & 1;
-        const uint64_t dv = slot ? dv1 : dv0;
-        // chunk c: dims 128c.. = atoms 2c, 2c+1 (A, MN-major); K step kk:
-        // tokens 16kk.. = +2048 B in A, +32 B in P
+        const int stage = t % kStages;
+        const uint64_t bv = stage == 0 ? dv[0] : (stage == 1 ? dv[1] : dv[2]);
+        // O[:, 256 hf + n] += P[:, 16 kk + k] V[16 kk + k, 256 hf + n]:
+        // A = P (K step +32 B), B = V MN-major (tokens +2048 B, dims 256
+        // = four atoms = +32768 B)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t d = tmem + kColO + 64u * (uint32_t)c;
-          const uint64_t a0 = dv + (uint64_t)(c * (2 * kAtomBytes >> 4));
-          if (t == 0) mma_set_elect(d, a0, dp, kIdescPV);
-          else mma_acc_elect(d, a0, dp, kIdescPV);
-          mma_acc_elect(d, a0 + 128, dp + 2, kIdescPV);
-          mma_acc_elect(d, a0 + 256, dp + 4, kIdescPV);
-          mma_acc_elect(d, a0 + 384, dp + 6, kIdescPV);
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t d = o0 + 256u * (uint32_t)hf;
+            const uint64_t a = dp + (uint64_t)(2 * kk);
+            const uint64_t bb = bv + (uint64_t)(128 * kk + 2048 * hf);
+            if (t == 0 && kk == 0) mma_set_elect(d, a, bb, kIdescPV);
+            else mma_acc_elect(d, a, bb, kIdescPV);
+          }
         }
-        commit_elect(BAR(BAR_KVE + slot));
+        commit_elect(BAR(BAR_KVE + stage));
         commit_elect(BAR(BAR_PVD));
         if (lane == 0 && t < 8) SMLA_TRACE_EV(16 + t);
       }
     }
     // drain: every MMA this warp issued has completed before teardown
-    // (each warp has its own completion barrier)
     commit_elect(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2));
     mbar_wait(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2), 0);
   } else {
     // ------------------------------------------------------------ softmax
-    const int h = 16 * warp + (lane & 15);   // head row of this thread
-    const int half = lane >> 4;              // tokens [32*half, 32*half+32)
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    // Thread (warp w, lane t) owns head h = 16w + t%16; lanes t and t+16 hold
+    // tokens [0,32) and [32,64) of a tile and dims [0,256) / [256,512) of O.
+    const int h = 16 * warp + (lane & 15);
+    const int half = lane >> 4;
+    const uint32_t q_lanes = (uint32_t)(32 * warp) << 16;            // Q / S rows
+    const uint32_t o_lanes = (uint32_t)(32 * warp + kLaneO) << 16;   // O rows
+    {  // the query row into tensor memory: dims [288 half, 288 half + 288),
+       // read from the copy staged in shared memory (row-major [64][576])
+      bool okq = mbar_wait(BAR(BAR_QS), 0);
+      if (okq) {
+        const uint8_t* qrow = smem + kSmemKV + 2 * kTileBytes + h * kRowBytesBf16 + half * 576;
+#pragma unroll 1
+        for (int c = 0; c < 9; ++c) {
+          uint32_t r[16];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qrow + c * 64 + u * 16);
+            r[4 * u] = v.x; r[4 * u + 1] = v.y; r[4 * u + 2] = v.z; r[4 * u + 3] = v.w;
+          }
+          tmem_st_16x32bx2_x16(tmem + q_lanes + kColQ + 16u * (uint32_t)c, r);  // second half at +144
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_QT));
+    }
     // l_run: sum of the probabilities as fp32 (gives lse); l_pv: the same sum
     // of the bf16-rounded probabilities the PV MMA used (normalises out, so
     // the output weights sum to one exactly).  fp8 rows fold the row scale
@@ -687,11 +758,13 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     bool aborted = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1, rs = i % kRing;
-      const bool f1 = !mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_IXF + rs), (i / kRing) & 1);
-      if (group_any(f1, 2, 128)) { aborted = true; break; }
+      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_IXF + rs), (i / kRing) & 1)) {
+        aborted = true;
+      }
+      if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
       tc_fence_after();
       float s[32];
-      tmem_ld_16x32bx2_x32(tmem + lane_base + kColS + 64u * (uint32_t)sb, s);
+      tmem_ld_16x32bx2_x32(tmem + q_lanes + kColS + 64u * (uint32_t)sb, s);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -739,24 +812,23 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         }
       }
       // P buffer and O are free once PV(i-1) has completed
-      const bool f2 = i >= 1 ? !mbar_wait(BAR(BAR_PVD), (i - 1) & 1) : false;
-      if (group_any(f2, 2, 128)) { aborted = true; break; }
+      if (i >= 1 && !mbar_wait(BAR(BAR_PVD), (i - 1) & 1)) aborted = true;
+      if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
       tc_fence_after();
+      // rescale this head's O row by alpha (O rows of the warp: lanes 16-31
+      // of its quarter; lane t and t+16 hold dims [0,256) and [256,512))
       const bool resc = need && i >= 1 && m_run > -INFINITY;
-      if (group_any(resc, 2, 128)) {
-        if (half == 0) s_alpha[h] = resc ? alpha : 1.f;
-        named_bar_sync(2, 128);
-        // O^T lanes are dims, columns are heads: scale column k by alpha[k]
+      if (__any_sync(0xffffffffu, resc)) {
+        const float f = resc ? alpha : 1.f;
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
           float o[32];
-          const uint32_t ta = tmem + lane_base + kColO + 32u * (uint32_t)c;
-          tmem_ld_32x32b_x32(ta, o);
+          const uint32_t ta = tmem + o_lanes + 32u * (uint32_t)c;
+          tmem_ld_16x32bx2_x32_h256(ta, o);
           tmem_wait_ld();
-          const float* al = s_alpha + (c & 1) * 32;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= al[k];
-          tmem_st_32x32b_x32(ta, o);
+          for (int k = 0; k < 32; ++k) o[k] *= f;
+          tmem_st_16x32bx2_x32_h256(ta, o);
         }
         tmem_wait_st();
       }
@@ -777,76 +849,66 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     }
     // ---------------------------------------------------------- epilogue
     if (!aborted && ntiles > 0) {
-      const bool f = !mbar_wait(BAR(BAR_PVD), (ntiles - 1) & 1);
-      aborted = group_any(f, 2, 128);
+      if (!mbar_wait(BAR(BAR_PVD), (ntiles - 1) & 1)) aborted = true;
+      aborted = __any_sync(0xffffffffu, aborted);
       tc_fence_after();
     }
     if (threadIdx.x == 0) SMLA_TRACE_EV(3);
     if (!aborted) {
-      float* s_invl = reinterpret_cast<float*>(smem + kEpiInvl);
-      float* s_lse = reinterpret_cast<float*>(smem + kEpiLse);
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       const bool any = l_tot > 0.f;
-      if (half == 0) {
-        s_invl[h] = any ? 1.f / l_nrm : 0.f;
-        s_lse[h] = any ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
-      }
-      named_bar_sync(2, 128);
+      const float inv_l = any ? 1.f / l_nrm : 0.f;
+      const float lse_h = any ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
       const bool direct = p.nsplit == 1;
-      // stage [64 heads][512 dims] in the (now idle) KV buffers
-      __nv_bfloat16* st_bf = reinterpret_cast<__nv_bfloat16*>(smem + kSmemKV);
-      float* st_f = reinterpret_cast<float*>(smem + kSmemKV);
+      const size_t part = (size_t)b * p.nsplit + split;
+      // Stage this warp's 16 head rows in shared memory (the idle KV stages)
+      // with a 16-byte pad per row, which makes the 16-byte stores of a warp
+      // conflict-free, then write each row with one bulk copy.
+      const uint32_t row_bytes = direct ? kDv * 2 : kDv * 4;
+      const uint32_t stride = row_bytes + 16;
+      uint8_t* srow = smem + kSmemKV + (size_t)h * stride;
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
         float o[32];
         if (ntiles > 0) {
-          tmem_ld_32x32b_x32(tmem + lane_base + kColO + 32u * (uint32_t)c, o);
+          tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int k = 0; k < 32; ++k) o[k] = 0.f;
         }
-        const int dim = (c >> 1) * 128 + 32 * warp + lane;
-        const int h0 = (c & 1) * 32;
-        float il[32];
-#pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          const float4 v4 = *reinterpret_cast<const float4*>(s_invl + h0 + k);
-          il[k] = v4.x; il[k + 1] = v4.y; il[k + 2] = v4.z; il[k + 3] = v4.w;
-        }
+        const int d0 = half * 256 + c * 32;   // this thread's 32 dims
         if (direct) {
+          uint4* dst = reinterpret_cast<uint4*>(srow + d0 * 2);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) st_bf[(h0 + k) * kDv + dim] = __float2bfloat16_rn(o[k] * il[k]);
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(pack_bf16x2(o[8 * u] * inv_l, o[8 * u + 1] * inv_l),
+                                pack_bf16x2(o[8 * u + 2] * inv_l, o[8 * u + 3] * inv_l),
+                                pack_bf16x2(o[8 * u + 4] * inv_l, o[8 * u + 5] * inv_l),
+                                pack_bf16x2(o[8 * u + 6] * inv_l, o[8 * u + 7] * inv_l));
         } else {
+          float4* dst = reinterpret_cast<float4*>(srow + d0 * 4);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) st_f[(h0 + k) * kDv + dim] = o[k] * il[k];
+          for (int u = 0; u < 8; ++u)
+            dst[u] = make_float4(o[4 * u] * inv_l, o[4 * u + 1] * inv_l, o[4 * u + 2] * inv_l,
+                                 o[4 * u + 3] * inv_l);
         }
       }
       fence_proxy_async_smem();
-      named_bar_sync(2, 128);
-      if (threadIdx.x == 0) {
-        SMLA_TRACE_EV(4);
-        if (direct) {
-          uint8_t* dst = reinterpret_cast<uint8_t*>(p.out + (size_t)b * kH * kDv);
-          for (int k = 0; k < 2; ++k)
-            bulk_store_s2g(dst + k * 32768, sbase + kSmemKV + k * 32768, 32768u);
-        } else {
-          const size_t part = (size_t)b * p.nsplit + split;
-          uint8_t* dst = reinterpret_cast<uint8_t*>(p.part_o + part * kH * kDv);
-          for (int k = 0; k < 4; ++k)
-            bulk_store_s2g(dst + k * 32768, sbase + kSmemKV + k * 32768, 32768u);
-        }
+      __syncwarp();
+      if (half == 0) {
+        uint8_t* gdst = direct ? reinterpret_cast<uint8_t*>(p.out + ((size_t)b * kH + h) * kDv)
+                               : reinterpret_cast<uint8_t*>(p.part_o + (part * kH + h) * kDv);
+        bulk_store_s2g(gdst, smem_u32(srow), row_bytes);
         bulk_commit();
       }
       if (half == 0) {
-        if (direct) p.lse[(size_t)b * kH + h] = s_lse[h];
-        else p.part_lse[((size_t)b * p.nsplit + split) * kH + h] = s_lse[h];
-      }
-      if (threadIdx.x == 0) {
+        if (direct) p.lse[(size_t)b * kH + h] = lse_h;
+        else p.part_lse[part * kH + h] = lse_h;
         bulk_wait_all();
-        SMLA_TRACE_EV(5);
       }
+      if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     }
     tc_fence_before();
   }
@@ -945,37 +1007,6 @@ static size_t partial_bytes(int batch, int nsplit) {
   return ((o + l + 255) / 256) * 256;
 }
 
-// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
-// point (no link against libcuda).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-// 2-D bf16 tensor [outer][inner] with rows `row_bytes` apart; box
-// box_inner x box_outer elements, 128-byte swizzle, zero fill out of range.
-static bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                           uint32_t box_inner, uint32_t box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // The shared-memory opt-in is set once per device (an idempotent call, so a
 // race between threads is harmless); later calls, including calls made
 // while a stream is being captured into a CUDA graph, skip it.
@@ -1023,7 +1054,6 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   }
   SplitParams prm;
   memset(&prm, 0, sizeof(prm));
-  if (!encode_bf16_2d(&prm.tmap_q, q, kDqk, (uint64_t)shape->batch * kH, kRowBytesBf16, 64, 64)) return SMLA_ERR_CUDA;
   prm.q = static_cast<const uint8_t*>(q);
   prm.kv = static_cast<const uint8_t*>(kv_cache);
   prm.kv_row_scale = kv_row_scale;
