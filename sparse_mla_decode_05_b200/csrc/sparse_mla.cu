@@ -67,22 +67,28 @@ constexpr int kRowBytesFp8 = kDqk;                  // 576
 // shared memory map (offsets from the 1024-aligned dynamic shared base)
 constexpr int kStages = 3;                          // KV tile stages
 constexpr int kSmemKV = 0;                          // KV  [3 stages][9 atoms][64 tok][128 B]
-constexpr int kSmemP = kSmemKV + kStages * kTileBytes;  // P [64 heads][64 tok] bf16 (K-major)
-constexpr int kSmemAux = kSmemP + 64 * 128;
+// P(t) [64 heads][64 tok] bf16 (K-major) takes the place of the rope atom of
+// the stage that holds tile t: S(t) has read that atom by the time P(t) is
+// written, PV(t) reads the rest of the stage, and the stage is refilled only
+// after PV(t).  Each stage thus carries its own P buffer.
+constexpr int kAtomP = kAtoms - 1;
+constexpr int kSmemAux = kSmemKV + kStages * kTileBytes;
 constexpr int kRing = 4;                            // resolved-row ring depth (tiles)
 // barrier indices
 constexpr int BAR_KVF = 0;                          // [kStages] tile landed
 constexpr int BAR_KVE = BAR_KVF + kStages;          // [kStages] tile consumed (PV done)
 constexpr int BAR_SF = BAR_KVE + kStages;           // [2] S(t) in TMEM
 constexpr int BAR_SE = BAR_SF + 2;                  // [2] S(t) read by the softmax
-constexpr int BAR_PF = BAR_SE + 2;                  // P(t) written
-constexpr int BAR_PVD = BAR_PF + 1;                 // PV(t) done
-constexpr int BAR_FIN = BAR_PVD + 1;                // drain, S issuer
+constexpr int BAR_PF = BAR_SE + 2;                  // [kStages] P(t) written (per stage)
+constexpr int BAR_PVD = BAR_PF + kStages;           // [2] PV(t) done (by tile parity)
+constexpr int BAR_FIN = BAR_PVD + 2;                // drain, S issuer
 constexpr int BAR_FIN2 = BAR_FIN + 1;               // drain, PV issuer
 constexpr int BAR_QT = BAR_FIN2 + 1;                // query written to TMEM
 constexpr int BAR_QS = BAR_QT + 1;                  // query staged in shared memory
-constexpr int BAR_IXF = BAR_QS + 1;                 // [kRing] rows resolved
-constexpr int BAR_IXE = BAR_IXF + kRing;            // [kRing] rows consumed
+constexpr int BAR_PVI = BAR_QS + 1;                 // [2] PV(t) issued (by tile parity)
+constexpr int BAR_IXF = BAR_PVI + 2;                // [kRing] rows resolved
+constexpr int BAR_IXS = BAR_IXF + kRing;            // [kRing] fp8 row scales resolved
+constexpr int BAR_IXE = BAR_IXS + kRing;            // [kRing] rows consumed
 constexpr int kNumBars = BAR_IXE + kRing;
 constexpr int kAuxBars = kSmemAux;
 constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
@@ -475,19 +481,21 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(BAR(BAR_KVF + s), kFp8 ? kLoad / 32 : kLoad);  // fp8: loader warps; bf16: async copies
       mbar_init(BAR(BAR_KVE + s), 1);
+      mbar_init(BAR(BAR_PF + s), 4);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(BAR_SF + s), 1);
       mbar_init(BAR(BAR_SE + s), 4);
+      mbar_init(BAR(BAR_PVD + s), 1);
+      mbar_init(BAR(BAR_PVI + s), 1);
     }
-    mbar_init(BAR(BAR_PF), 4);
-    mbar_init(BAR(BAR_PVD), 1);
     mbar_init(BAR(BAR_FIN), 1);
     mbar_init(BAR(BAR_FIN2), 1);
     mbar_init(BAR(BAR_QT), 4);
     mbar_init(BAR(BAR_QS), 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(BAR(BAR_IXF + r), 1);
+      mbar_init(BAR(BAR_IXS + r), 1);
       mbar_init(BAR(BAR_IXE + r), kLoad / 32 + 4);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -555,14 +563,17 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       const int i3_0 = idx_at(t + 3 * S, lane), i3_1 = idx_at(t + 3 * S, lane + 32);
       const bool fail = t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1);
       if (__any_sync(0xffffffffu, fail)) break;  // warp-uniform exit
+      // rows first (the loaders need only them), then the row scales
       s_row[rs * 64 + lane] = r0_0;
       s_row[rs * 64 + lane + 32] = r0_1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_IXF + rs));
       if (kFp8) {
         s_rsc[rs * 64 + lane] = c0_0;
         s_rsc[rs * 64 + lane + 32] = c0_1;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(BAR_IXF + rs));
+      if (lane == 0) mbar_arrive(BAR(BAR_IXS + rs));
       if (lane == 0 && t < 4) SMLA_TRACE_EV(58 + t);
       r0_0 = r1_0; r0_1 = r1_1;
       c0_0 = c1_0; c0_1 = c1_1;
@@ -665,9 +676,12 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       if (lane == 0) SMLA_TRACE_EV(2);
       for (int t = 0; ok && t < ntiles; ++t) {
         const int stage = t % kStages, sb = t & 1;
-        // S(t) reuses the S buffer of S(t-2): its softmax must have read it
+        // S(t) reuses the S buffer of S(t-2): its softmax must have read it.
+        // It also waits until PV(t-2) has been issued, which keeps the
+        // tensor-core queue in the order S(t-1), PV(t-2), S(t), PV(t-1):
+        // issued earlier, S(t) would delay PV(t-2) and with it the softmax.
         if (t >= 2) {
-          ok = wait_all(BAR(BAR_SE + sb), ((t >> 1) - 1) & 1);
+          ok = wait_all(BAR(BAR_SE + sb), ((t >> 1) - 1) & 1) && wait_all(BAR(BAR_PVI + sb), ((t >> 1) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
         }
@@ -691,14 +705,15 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       uint64_t dv[kStages];
 #pragma unroll
       for (int s = 0; s < kStages; ++s) dv[s] = sw128_desc(sbase + kSmemKV + s * kTileBytes, kAtomBytes, 1024);
-      const uint64_t dp = sw128_desc(sbase + kSmemP, 16, 1024);
       const uint32_t o0 = tmem + (kLaneO << 16);
       for (int t = 0; ok && t < ntiles; ++t) {
-        ok = wait_all(BAR(BAR_PF), t & 1);
+        const int stage = t % kStages;
+        ok = wait_all(BAR(BAR_PF + stage), (t / kStages) & 1);
         if (!ok) break;
         tc_fence_after();
-        const int stage = t % kStages;
         const uint64_t bv = stage == 0 ? dv[0] : (stage == 1 ? dv[1] : dv[2]);
+        // P(t) sits in the stage's rope atom
+        const uint64_t dp = sw128_desc(sbase + kSmemKV + stage * kTileBytes + kAtomP * kAtomBytes, 16, 1024);
         // O[:, 256 hf + n] += P[:, 16 kk + k] V[16 kk + k, 256 hf + n]:
         // A = P (K step +32 B), B = V MN-major (tokens +2048 B, dims 256
         // = four atoms = +32768 B)
@@ -714,7 +729,9 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
           }
         }
         commit_elect(BAR(BAR_KVE + stage));
-        commit_elect(BAR(BAR_PVD));
+        commit_elect(BAR(BAR_PVD + (t & 1)));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(BAR_PVI + (t & 1)));
         if (lane == 0 && t < 8) SMLA_TRACE_EV(16 + t);
       }
     }
@@ -758,7 +775,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     bool aborted = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1, rs = i % kRing;
-      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_IXF + rs), (i / kRing) & 1)) {
+      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1)) {
         aborted = true;
       }
       if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
@@ -811,14 +828,16 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
           lsum_pv += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
         }
       }
-      // P buffer and O are free once PV(i-1) has completed
-      if (i >= 1 && !mbar_wait(BAR(BAR_PVD), (i - 1) & 1)) aborted = true;
-      if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
-      tc_fence_after();
-      // rescale this head's O row by alpha (O rows of the warp: lanes 16-31
-      // of its quarter; lane t and t+16 hold dims [0,256) and [256,512))
+      // Rescale this head's O row by alpha (O rows of the warp: lanes 16-31
+      // of its quarter; lane t and t+16 hold dims [0,256) and [256,512)).
+      // Only then must PV(i-1) have completed.  PVD[(i-1)&1] cannot be more
+      // than one phase behind: tile i was loaded after PV(i-3) released its
+      // stage, and PV(i+1) needs this warp's P(i+1).
       const bool resc = need && i >= 1 && m_run > -INFINITY;
       if (__any_sync(0xffffffffu, resc)) {
+        if (!mbar_wait(BAR(BAR_PVD + ((i - 1) & 1)), ((i - 1) >> 1) & 1)) aborted = true;
+        if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
+        tc_fence_after();
         const float f = resc ? alpha : 1.f;
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -835,7 +854,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       l_run = l_run * alpha + lsum;
       l_pv = kFp8 ? l_run : l_pv * alpha + lsum_pv;
       m_run = m_use;
-      const uint32_t prow = sbase + kSmemP;
+      const uint32_t prow = sbase + kSmemKV + (i % kStages) * kTileBytes + kAtomP * kAtomBytes;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         st_shared_v4(prow + sw128_off(h, half * 4 + q4),
@@ -844,12 +863,14 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(BAR_PF));
+      if (lane == 0) mbar_arrive(BAR(BAR_PF + i % kStages));
       if (threadIdx.x == 0 && i < 8) SMLA_TRACE_EV(32 + i);
     }
     // ---------------------------------------------------------- epilogue
     if (!aborted && ntiles > 0) {
-      if (!mbar_wait(BAR(BAR_PVD), (ntiles - 1) & 1)) aborted = true;
+      // PV(n-2) then PV(n-1): each wait is at most one phase ahead
+      if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + (ntiles & 1)), ((ntiles - 2) >> 1) & 1)) aborted = true;
+      if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1)) aborted = true;
       aborted = __any_sync(0xffffffffu, aborted);
       tc_fence_after();
     }
