@@ -7,9 +7,10 @@ One step = one sparse_mla_decode call (split kernel + combine when the plan
 splits) over one batch of the headline workload, inputs resident in HBM.
 L2 is flushed (a write of 2x the L2 size) before every timed step, outside
 the timed region; each step is timed with CUDA events on the launching
-stream.  With N > 1 (torchrun) every rank runs an independent replica of the
-workload (the op shards over batch with no exchange): weak scaling, time =
-max over ranks.  Rank 0 prints one JSON line.
+stream.  With N > 1 (torchrun) every rank runs the workload on its own batch
+of sequences (the op shards over batch with no exchange step; rank r draws
+its batch with inputs.shard_seed): weak scaling, value = bytes of all ranks
+over the max-over-ranks time.  Rank 0 prints one JSON line.
 
 Keys beyond the base contract:
   roofline     dominant kernel (the split kernel) vs the measured HBM peak
@@ -110,6 +111,17 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- helpers
+def reduce_over_ranks(x: float, op: str, device) -> float:
+    """max or sum of a host float over all ranks of the default process group
+    (the value itself without one)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def to_dev(w: inputs.Workload, dev):
     return dict(q=w.q.to(dev), kv=w.kv.to(dev), indices=w.indices.to(dev),
                 kv_row_scale=None if w.kv_row_scale is None else w.kv_row_scale.to(dev),
@@ -229,13 +241,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     peak_gbs, peak_tf, peak_tf_sus, peak_src = load_peaks()
-    w = inputs.make_config(args.workload)
+    w = inputs.make_config(args.workload, seed=inputs.shard_seed(args.workload, rank))
     alg_bytes = inputs.algorithmic_bytes(w)
     alg_flops = inputs.algorithmic_flops(w)
     config = {"workload": f"{args.workload}: {inputs.CONFIG_DESCRIPTIONS[args.workload]}", "batch": w.batch,
               "topk": w.topk, "heads": 64, "d_qk": 576, "d_v": 512, "kv_dtype": w.kv_format,
               "paged": w.page_size > 0, "l2": "flushed before every timed step (2x L2 write, untimed)",
-              "parallelism": f"replicas x{args.gpus} (weak)" if args.gpus > 1 else "single GPU"}
+              "parallelism": f"batch shards x{world} (weak, no collective)" if world > 1 else "single GPU"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -284,13 +296,9 @@ def main():
     t_clk1 = time.time()
     t_wall = time.perf_counter() - t_wall0
     clocks = clk.summary(t_clk0, t_clk1)
-    ms = float(np.mean(times))
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
-    value = alg_bytes * world / (ms * 1e-3) / 1e9
+    ms = reduce_over_ranks(float(np.mean(times)), "max", dev)
+    job_bytes = reduce_over_ranks(alg_bytes, "sum", dev)
+    value = job_bytes / (ms * 1e-3) / 1e9
 
     # --- dominant kernel (split) and combine, each timed on its own
     sp, cb = time_split_breakdown(r, max(10, args.steps // 2), flush, stream)
@@ -328,19 +336,14 @@ def main():
         hlse.copy_(e2e_plan.lse, non_blocking=True)
 
     e2e_times = time_device(e2e_step, max(10, args.steps // 2), 3, flush, stream)
-    e2e_ms = float(np.mean(e2e_times))
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e = {"value": alg_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    e2e_ms = reduce_over_ranks(float(np.mean(e2e_times)), "max", dev)
+    e2e = {"value": job_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     assert api.device_error() == 0, "device error word set"
 
     # --- every workload at 1 GPU (rank 0 only)
     per_config = None
-    if rank == 0 and not args.no_per_config:
+    if rank == 0 and world == 1 and not args.no_per_config:
         per_config = []
         for name in inputs.CONFIG_NAMES:
             wc = w if name == args.workload else inputs.make_config(name)

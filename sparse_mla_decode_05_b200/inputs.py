@@ -215,6 +215,18 @@ def make_config(name: str, seed: int | None = None) -> Workload:
     raise KeyError(name)
 
 
+def shard_seed(name: str, rank: int) -> int | None:
+    """Seed of rank ``rank``'s batch of workload ``name`` when the step runs
+    as independent per-GPU batches (the op shards over sequences): rank 0
+    keeps the workload's own seed (None), rank r > 0 draws a distinct one."""
+    if rank < 0:
+        raise ValueError("rank must be >= 0")
+    if rank == 0:
+        return None
+    base = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005}[name]
+    return base + 100_000 * rank
+
+
 def algorithmic_bytes(w: Workload) -> int:
     """Bytes the step must move at minimum: valid gathered rows (row bytes,
     plus the 4-byte row scale for fp8 pools), q, out, lse, the index list and
