@@ -163,6 +163,44 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
  * the word was non-zero, SMLA_OK if zero, SMLA_ERR_CUDA on a copy failure. */
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
+/* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:
+ * 24 MiB, enough for batch * nsplit <= 191 split partials (131,328 bytes
+ * each).  Every split count the planner picks on a 148-SM B200 fits (it keeps
+ * batch * nsplit <= 148). */
+#define SMLA_STATIC_SCRATCH_BYTES ((size_t)24 << 20)
+
+/* The whole decode step, for callers that cannot allocate device memory.
+ * The source pages have no counterpart to this entry point.
+ *
+ * It computes exactly what sparse_mla_decode computes, with the same
+ * arguments except the workspace.  When the plan splits top-k (nsplit > 1),
+ * the split partials go to a scratch buffer of SMLA_STATIC_SCRATCH_BYTES
+ * that the library holds in device memory as a static array: one per
+ * device, created when the library's device code is loaded.  Neither this
+ * call nor the library allocates or frees anything.
+ *
+ * - Size limit.  A shape whose partials would not fit is rejected with
+ *   SMLA_ERR_WORKSPACE before any launch.  With shape->nsplit > 0 the check
+ *   is made before any CUDA call.  Use sparse_mla_decode with your own
+ *   workspace for such shapes.
+ * - Zeroing.  Every split writes its whole partial (an empty split writes
+ *   o = 0, lse = -inf), so nothing in the scratch has to start at zero and
+ *   nothing is cleared.
+ * - First call.  The first call on a device looks up the scratch address
+ *   with cudaGetSymbolAddress, with that device current, and keeps it.  A
+ *   failed lookup returns SMLA_ERR_CUDA.  If you capture streams, make one
+ *   call on each device before capturing, so that this set-up is done.
+ * - Races.  All calls on one device share the one scratch buffer.  Calls
+ *   that can overlap in time (different streams, different host threads
+ *   without ordering) race on it and corrupt each other's results.  Issue
+ *   them on one stream, or otherwise order them.
+ *
+ * Errors and validation are as for sparse_mla_decode. */
+smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void* q, const void* kv_cache,
+                                             const float* kv_row_scale, const int32_t* page_table,
+                                             const int32_t* indices, float scale, void* out, float* lse,
+                                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif

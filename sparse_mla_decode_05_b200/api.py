@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
     lib.sparse_mla_combine.argtypes = [I32, I32, I32, I32, P, P, P, P, P]
     lib.sparse_mla_get_device_error.restype = I32
     lib.sparse_mla_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    lib.sparse_mla_decode_static_scratch.restype = I32
+    lib.sparse_mla_decode_static_scratch.argtypes = [SP, P, P, P, P, P, F32, P, P, P]
     return lib
 
 
@@ -131,6 +133,27 @@ def decode(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=None, 
                                _stream(dev))
     if st != 0:
         raise SmlaError(st, "sparse_mla_decode")
+    return out, lse
+
+
+# Scratch size of decode_static_scratch (SMLA_STATIC_SCRATCH_BYTES).
+STATIC_SCRATCH_BYTES = 24 << 20
+
+
+def decode_static_scratch(q, kv, indices, scale: float, out, lse, *, kv_row_scale=None, page_table=None,
+                          page_size: int = 0, nsplit: int = 0):
+    """sparse_mla_decode_static_scratch: the decode step into caller-given
+    ``out`` [B,64,512] bf16 and ``lse`` [B,64] fp32, with the split partials
+    in the library's own static device scratch (STATIC_SCRATCH_BYTES), for
+    callers that cannot allocate.  Calls that overlap in time on one device
+    share that scratch and race; issue them on one stream."""
+    _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size)
+    shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
+    st = lib.sparse_mla_decode_static_scratch(ctypes.byref(shape), _ptr(q), _ptr(kv), _ptr(kv_row_scale),
+                                              _ptr(page_table), _ptr(indices), float(scale), _ptr(out),
+                                              _ptr(lse), _stream(q.device))
+    if st != 0:
+        raise SmlaError(st, "sparse_mla_decode_static_scratch")
     return out, lse
 
 

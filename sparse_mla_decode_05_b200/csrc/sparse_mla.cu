@@ -49,6 +49,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "sparse_mla.h"
 
 namespace smla {
@@ -154,6 +156,10 @@ struct SplitParams {
 };
 
 __device__ unsigned int g_error_word = 0;
+
+// Scratch for sparse_mla_decode_static_scratch: split partials for callers
+// that cannot allocate (one buffer per device, shared by all such calls).
+static __device__ __align__(256) unsigned char g_static_scratch[SMLA_STATIC_SCRATCH_BYTES];
 
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -1107,6 +1113,23 @@ static smla_status run_combine(int batch, int nsplit, const float* part_o, const
   return cudaGetLastError() == cudaSuccess ? SMLA_OK : SMLA_ERR_CUDA;
 }
 
+// Device address of g_static_scratch on the current device, looked up once
+// per device (with that device current) and kept.
+static smla_status static_scratch_address(void** ptr) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SMLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return SMLA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return SMLA_OK;
+}
+
 }  // namespace smla
 
 // ============================================================ C ABI
@@ -1171,6 +1194,29 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
       !smla::aligned(lse, 4))
     return SMLA_ERR_INVALID_ARG;
   return smla::run_combine(batch, nsplit, partial_o, partial_lse, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void* q, const void* kv_cache,
+                                             const float* kv_row_scale, const int32_t* page_table,
+                                             const int32_t* indices, float scale, void* out, float* lse,
+                                             void* stream) {
+  smla_status st = smla::validate_shape(shape);
+  if (st != SMLA_OK) return st;
+  // split count and scratch need: no CUDA call when the caller fixes nsplit
+  const int n = shape->nsplit > 0 ? smla::plan_nsplit(shape, 0) : smla::plan_nsplit(shape, smla::device_sm_count());
+  if (shape->nsplit == 0 && smla::device_sm_count() <= 0) return SMLA_ERR_CUDA;
+  const size_t need = n > 1 ? smla::partial_bytes(shape->batch, n) : 0;
+  if (need > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    st = smla::static_scratch_address(&scratch);
+    if (st != SMLA_OK) return st;
+  }
+  // the planned count, fixed, so the launch uses exactly the checked size
+  smla_shape fixed = *shape;
+  fixed.nsplit = n;
+  return sparse_mla_decode(&fixed, q, kv_cache, kv_row_scale, page_table, indices, scale, out, lse, scratch,
+                           need, stream);
 }
 
 smla_status sparse_mla_get_device_error(uint32_t* code) {
