@@ -23,9 +23,11 @@ Keys beyond the base contract:
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import time
@@ -111,6 +113,26 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- helpers
+KERNEL_SOURCE = os.path.join(ROOT, "sparse_mla_decode_05_b200", "csrc", "sparse_mla.cu")
+
+
+def kernel_traffic(workload: str):
+    """DRAM bytes (read + write) per launch of the split kernel on `workload`,
+    from the committed ncu summary profiles/smla_split_kernel_<workload>_dram.md;
+    None when there is none or it was taken on another kernel source."""
+    path = os.path.join(ROOT, "profiles", f"smla_split_kernel_{workload}_dram.md")
+    try:
+        text = open(path).read()
+        src = hashlib.sha256(open(KERNEL_SOURCE, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel source sha256: `?([0-9a-f]{64})", text)
+    m_b = re.search(r"dram bytes per launch: `?(\d+)", text)
+    if not (m_sha and m_b) or m_sha.group(1) != src:
+        return None
+    return int(m_b.group(1))
+
+
 def reduce_over_ranks(x: float, op: str, device) -> float:
     """max or sum of a host float over all ranks of the default process group
     (the value itself without one)."""
@@ -157,7 +179,7 @@ class Runner:
 
     @property
     def launches_per_step(self):
-        return 1 + (1 if self.nsplit > 1 else 0)
+        return 1 + (1 if self.nsplit > 1 and not self.plan.clustered else 0)
 
 
 def time_device(fn, steps, warmup, flush, stream):
@@ -303,11 +325,12 @@ def main():
     # --- dominant kernel (split) and combine, each timed on its own
     sp, cb = time_split_breakdown(r, max(10, args.steps // 2), flush, stream)
     sp_ms = float(np.mean(sp))
-    cb_ms = float(np.mean(cb)) if r.nsplit > 1 else 0.0
+    cb_ms = float(np.mean(cb)) if r.nsplit > 1 and not r.plan.clustered else 0.0
     achieved = alg_bytes / (sp_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak_gbs, "unit": "GB/s", "frac": achieved / peak_gbs,
-            "traffic": None, "kernel": "smla_split_kernel", "peak_source": f"{peak_src} (burst copy)",
+            "traffic": kernel_traffic(args.workload), "algorithmic_bytes": alg_bytes, "kernel": "smla_split_kernel", "peak_source": f"{peak_src} (burst copy)",
             "split_kernel_us": sp_ms * 1e3, "combine_kernel_us": cb_ms * 1e3, "nsplit": r.nsplit,
+            "split_reduction": "cluster (on chip)" if r.plan.clustered else ("partials + combine" if r.nsplit > 1 else "none"),
             "roofline_us": roofline_us(w, peak_gbs, peak_tf),
             "frac_of_step_roofline": roofline_us(w, peak_gbs, peak_tf) / (ms * 1e3),
             "frac_vs_nominal_8TBps": achieved / 8000.0}
@@ -355,6 +378,7 @@ def main():
             ab = inputs.algorithmic_bytes(wc)
             rl = roofline_us(wc, peak_gbs, peak_tf)
             per_config.append({"workload": name, "batch": wc.batch, "topk": wc.topk, "nsplit": rc.nsplit,
+                               "clustered": rc.plan.clustered,
                                "us_per_call": med, "p10_us": p10, "p90_us": p90,
                                "gbs": ab / (med * 1e-6) / 1e9, "roofline_us": rl, "frac_roofline": rl / med,
                                "split_kernel_us": float(np.median(spc)) * 1e3,

@@ -100,9 +100,26 @@ int32_t sparse_mla_abi_version(void);
 const char* sparse_mla_status_string(smla_status status);
 
 /* Number of top-k splits the decode will use for `shape` on the current
- * device: a pure function of (batch, topk, shape->nsplit, SM count), so the
- * grid is fixed per batch bucket.  Returns 0 if `shape` is invalid. */
+ * device: a pure function of (batch, topk, shape->nsplit, SM count, cluster
+ * limit), so the grid is fixed per batch bucket.  Returns 0 if `shape` is
+ * invalid.
+ *
+ * With more than one split, sparse_mla_decode merges the splits in one of
+ * two ways (sparse_mla_plan_merge tells which).  When nsplit is a power of
+ * two no larger than 16 that the device can launch as a thread-block
+ * cluster, the CTAs of a sequence form a cluster: each writes its partial
+ * result to the workspace, the cluster synchronises, and each CTA reduces
+ * one block of output columns -- one kernel.  Otherwise each split writes
+ * a partial result and a second (combine) kernel merges them.  An automatic
+ * plan (shape->nsplit == 0) takes the largest such power of two for which
+ * all clusters are resident at once. */
 int32_t sparse_mla_plan_nsplit(const smla_shape* shape);
+
+/* How sparse_mla_decode merges the splits of `shape` on the current device:
+ * 0 = one split (nothing to merge), 1 = inside the split kernel (thread-block
+ * cluster, one launch), 2 = partials and the combine kernel (two launches).
+ * Returns -1 if `shape` is invalid. */
+int32_t sparse_mla_plan_merge(const smla_shape* shape);
 
 /* Bytes of device workspace sparse_mla_decode needs for `shape` (0 when the
  * plan uses one split).  Deterministic in the shape, so a workspace sized
@@ -110,7 +127,8 @@ int32_t sparse_mla_plan_nsplit(const smla_shape* shape);
  * Returns 0 for an invalid shape. */
 size_t sparse_mla_workspace_size(const smla_shape* shape);
 
-/* One decode step (split kernel + combine when the plan splits).
+/* One decode step: the split kernel, plus the combine kernel when the plan
+ * merges its splits through a second kernel (sparse_mla_plan_merge == 2).
  *   q            [B, 64, 576] bf16
  *   kv_cache     [num_kv_rows, 576] bf16, or uint8 e4m3fn codes
  *   kv_row_scale [num_kv_rows] fp32 for SMLA_KV_FP8_E4M3_ROWSCALE, else NULL
@@ -129,9 +147,11 @@ smla_status sparse_mla_decode(const smla_shape* shape, const void* q, const void
                               const int32_t* indices, float scale, void* out, float* lse,
                               void* workspace, size_t workspace_bytes, void* stream);
 
-/* The split kernel alone: the hot loop of sparse_mla_decode.
+/* The split kernel alone, always in its partials form (never the on-chip
+ * merge), with the split count sparse_mla_plan_nsplit gives.
  * With nsplit == 1 it writes out/lse directly (workspace unused).  With
- * nsplit > 1 it writes per-split partial results into the workspace:
+ * nsplit > 1 it writes per-split partial results into the workspace, which
+ * must hold B*nsplit*64*(512+1)*4 bytes rounded up to a multiple of 256:
  *   partial_o   = workspace                      [B, nsplit, 64, 512] fp32,
  *                 each split's output normalised by its own softmax sum
  *                 (0 when the split holds no valid entry)
@@ -164,25 +184,26 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
 /* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:
- * 24 MiB, enough for batch * nsplit <= 191 split partials (131,328 bytes
- * each).  Every split count the planner picks on a 148-SM B200 fits (it keeps
- * batch * nsplit <= 148). */
+ * 24 MiB, enough for batch * nsplit <= 190 split results (at most 132,096
+ * bytes each).  Every split count the planner picks on a 148-SM B200 fits
+ * (it keeps batch * nsplit <= 148). */
 #define SMLA_STATIC_SCRATCH_BYTES ((size_t)24 << 20)
 
 /* The whole decode step, for callers that cannot allocate device memory.
  * The source pages have no counterpart to this entry point.
  *
  * It computes exactly what sparse_mla_decode computes, with the same
- * arguments except the workspace.  When the plan splits top-k (nsplit > 1),
- * the split partials go to a scratch buffer of SMLA_STATIC_SCRATCH_BYTES
+ * arguments except the workspace.  When the plan has more than one split,
+ * the split results go to a scratch buffer of SMLA_STATIC_SCRATCH_BYTES
  * that the library holds in device memory as a static array: one per
  * device, created when the library's device code is loaded.  Neither this
  * call nor the library allocates or frees anything.
  *
- * - Size limit.  A shape whose partials would not fit is rejected with
- *   SMLA_ERR_WORKSPACE before any launch.  With shape->nsplit > 0 the check
- *   is made before any CUDA call.  Use sparse_mla_decode with your own
- *   workspace for such shapes.
+ * - Size limit.  A shape whose split results would not fit is rejected
+ *   with SMLA_ERR_WORKSPACE before any launch; when shape->nsplit fixes the
+ *   split count and even its partials (131,328 bytes per sequence and
+ *   split) cannot fit, before any CUDA call.  Use sparse_mla_decode with
+ *   your own workspace for such shapes.
  * - Zeroing.  Every split writes its whole partial (an empty split writes
  *   o = 0, lse = -inf), so nothing in the scratch has to start at zero and
  *   nothing is cleared.

@@ -49,6 +49,8 @@ def _load() -> ctypes.CDLL:
     lib.sparse_mla_status_string.argtypes = [I32]
     lib.sparse_mla_plan_nsplit.restype = I32
     lib.sparse_mla_plan_nsplit.argtypes = [SP]
+    lib.sparse_mla_plan_merge.restype = I32
+    lib.sparse_mla_plan_merge.argtypes = [SP]
     lib.sparse_mla_workspace_size.restype = SZ
     lib.sparse_mla_workspace_size.argtypes = [SP]
     lib.sparse_mla_decode.restype = I32
@@ -90,6 +92,12 @@ def shape_for(q, kv, indices, *, page_table=None, page_size: int = 0, nsplit: in
 
 def plan_nsplit(shape: SmlaShape) -> int:
     return lib.sparse_mla_plan_nsplit(ctypes.byref(shape))
+
+
+def plan_merge(shape: SmlaShape) -> int:
+    """0: one split; 1: splits merged inside the split kernel (cluster);
+    2: partials merged by the combine kernel."""
+    return lib.sparse_mla_plan_merge(ctypes.byref(shape))
 
 
 def workspace_size(shape: SmlaShape) -> int:
@@ -168,7 +176,8 @@ def decode_split(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=
         out = torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
     if lse is None:
         lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
-    ws_bytes = workspace_size(shape)
+    nplan = plan_nsplit(shape)
+    ws_bytes = partials_size(q.shape[0], nplan) if nplan > 1 else 0
     if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     n = ctypes.c_int32(0)
@@ -180,6 +189,13 @@ def decode_split(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=
     if st != 0:
         raise SmlaError(st, "sparse_mla_decode_split")
     return n.value, out, lse, workspace
+
+
+def partials_size(batch: int, nsplit: int) -> int:
+    """Workspace bytes sparse_mla_decode_split needs to hold the partials of
+    `nsplit` splits (fp32 O and lse), rounded up to 256."""
+    b = batch * nsplit * H * (D_V + 1) * 4
+    return (b + 255) // 256 * 256
 
 
 def partial_views(workspace, batch: int, nsplit: int):
@@ -229,6 +245,8 @@ class DecodePlan:
         self.shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
         dev = q.device
         self.nsplit = plan_nsplit(self.shape)
+        # the splits merge inside the split kernel (one launch, no combine)
+        self.clustered = plan_merge(self.shape) == 1
         self.out = out if out is not None else torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
         self.lse = lse if lse is not None else torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
         ws = workspace_size(self.shape)
@@ -241,7 +259,7 @@ class DecodePlan:
         self._args = (ctypes.byref(self.shape), _ptr(q), _ptr(kv), _ptr(kv_row_scale), _ptr(page_table),
                       _ptr(indices), float(scale), _ptr(self.out), _ptr(self.lse), wsp, wsn)
         self._split_args = self._args + (None,)
-        if self.nsplit > 1:
+        if self.nsplit > 1 and not self.clustered:
             po, pl = partial_views(self.workspace, q.shape[0], self.nsplit)
             self._combine_args = (q.shape[0], H, D_V, self.nsplit, _ptr(po), _ptr(pl), _ptr(self.out),
                                   _ptr(self.lse))
@@ -254,6 +272,9 @@ class DecodePlan:
             raise SmlaError(st, "sparse_mla_decode")
 
     def run_split(self, stream=None):
+        """The split kernel of run(): all of run() when the splits reduce on chip."""
+        if self.clustered:
+            return self.run(stream)
         st = lib.sparse_mla_decode_split(*self._split_args, self._stream if stream is None else stream)
         if st != 0:
             raise SmlaError(st, "sparse_mla_decode_split")

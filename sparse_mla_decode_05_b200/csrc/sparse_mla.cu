@@ -44,7 +44,6 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <stdint.h>
 #include <math.h>
 #include <string.h>
@@ -91,7 +90,9 @@ constexpr int BAR_PVI = BAR_QS + 1;                 // [2] PV(t) issued (by tile
 constexpr int BAR_IXF = BAR_PVI + 2;                // [kRing] rows resolved
 constexpr int BAR_IXS = BAR_IXF + kRing;            // [kRing] fp8 row scales resolved
 constexpr int BAR_IXE = BAR_IXS + kRing;            // [kRing] rows consumed
-constexpr int kNumBars = BAR_IXE + kRing;
+constexpr int BAR_RAW = BAR_IXE + kRing;            // [kStages] fp8 codes landed
+constexpr int BAR_CS1 = BAR_RAW + kStages;          // cluster: every split's blocks written
+constexpr int kNumBars = BAR_CS1 + 1;
 constexpr int kAuxBars = kSmemAux;
 constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
 constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
@@ -130,13 +131,16 @@ constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // warps 0-3 softmax/epilogue, 4 S-MMA issuer (+ TMEM allocator), 5 PV-MMA
 // issuer, 6-9 index resolvers (warp 6+k owns the tiles t = k mod 4), 10..
-// loaders (bf16 rows: four warps issuing 16-byte cp.async; fp8 rows: eight
-// warps that load, convert and store)
+// loaders: copy warps issuing 16-byte cp.async (bf16 rows: four warps; fp8
+// codes: two warps), then, for fp8 only, eight warps that convert the codes
+// to bf16 in place
 constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kIdxWarps = 4, kWarpLoad0 = kWarpIdx + kIdxWarps;
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kLoadWarps = kFp8 ? 8 : 4;
-  static constexpr int kLoadThreads = kLoadWarps * 32;
+  static constexpr int kCopyWarps = kFp8 ? 2 : 4;
+  static constexpr int kCvtWarps = kFp8 ? 8 : 0;
+  static constexpr int kCopyThreads = kCopyWarps * 32;
+  static constexpr int kLoadWarps = kCopyWarps + kCvtWarps;
   static constexpr int kThreads = (kWarpLoad0 + kLoadWarps) * 32;
 };
 
@@ -151,6 +155,7 @@ struct SplitParams {
   float* part_o;               // [B, nsplit, 64, 512]
   float* part_lse;             // [B, nsplit, 64]
   int batch, topk, nsplit, ntiles_total;
+  int cluster;                 // 1: the nsplit CTAs of a sequence form a cluster and reduce on chip
   int page_size, pages_per_seq;
   float scale_log2;            // scale * log2(e)
 };
@@ -245,11 +250,12 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                "r"(v.w)
                : "memory");
 }
-__device__ __forceinline__ uint4 ld_global_nc_v4(const void* p) {
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+               : "r"(addr)
+               : "memory");
   return v;
 }
 __device__ __forceinline__ float ex2(float x) {
@@ -263,13 +269,30 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
-// two fp8 e4m3fn codes (low byte first) -> packed bf16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t codes) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
-  const float lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-  const float hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-  return pack_bf16x2(lo, hi);
+// bf16x2 product, round to nearest even
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// Four fp8 e4m3fn codes (one 32-bit word, lowest byte first) -> two packed
+// bf16x2 words (codes 0,1 and 2,3), exact for every non-NaN code, with
+// integer and bf16x2 arithmetic only (the conversion instructions run at a
+// fraction of that rate).  Each code's sign goes to bit 15 and its exponent
+// and mantissa bits to bits 10..4 of a bf16, which then holds the code's
+// value times 2^-120: the exponent field is read with bias 127 instead of 7,
+// and a zero exponent field reads as a bf16 subnormal just as it reads as an
+// e4m3 subnormal.  One bf16 multiply by 2^120 (subnormal inputs are kept,
+// the product is exact) restores the value.  NaN codes come out finite.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  constexpr uint32_t kTwo120 = 0x7B807B80u;          // 2^120 in both bf16 halves
+  const uint32_t u0 = __byte_perm(w, 0, 0x4140);     // code 1 -> bits 23..16, code 0 -> bits 7..0
+  const uint32_t u1 = __byte_perm(w, 0, 0x4342);     // codes 3, 2
+  // (sign << 15) | (magnitude << 4) per half: 16 u + 240 (u & signs)
+  const uint32_t b0 = u0 * 16u + (u0 & 0x00800080u) * 240u;
+  const uint32_t b1 = u1 * 16u + (u1 & 0x00800080u) * 240u;
+  lo = bf16x2_mul(b0, kTwo120);
+  hi = bf16x2_mul(b1, kTwo120);
 }
 
 // ---- tcgen05 (5th-generation tensor cores, tensor memory)
@@ -438,6 +461,53 @@ __device__ __forceinline__ void bulk_store_s2g(void* gdst, uint32_t ssrc, uint32
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// ---- thread-block cluster (distributed shared memory)
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_v4f(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+// arrive (release at cluster scope) on an mbarrier of any CTA of the cluster
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with acquire at cluster scope (sees what the arriving CTAs
+// released); false and an error bit on time-out.
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cluster(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(&g_error_word, 1u);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// every thread of every CTA of the cluster (executed unconditionally by all)
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -454,7 +524,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 template <bool kFp8>
 __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     smla_split_kernel(const __grid_constant__ SplitParams p) {
-  constexpr int kLoad = Cfg<kFp8>::kLoadThreads;
+  constexpr int kCopy = Cfg<kFp8>::kCopyThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bars = sbase + kAuxBars;
@@ -485,7 +555,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     // Arrivals are per warp (the warp synchronises, one lane arrives), except
     // where a copy engine arrives: mbarrier arrivals are serialised.
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(BAR(BAR_KVF + s), kFp8 ? kLoad / 32 : kLoad);  // fp8: loader warps; bf16: async copies
+      // bf16: one arrival per copying thread (when its copies land); fp8:
+      // one per convert warp
+      mbar_init(BAR(BAR_KVF + s), kFp8 ? Cfg<kFp8>::kCvtWarps : kCopy);
+      mbar_init(BAR(BAR_RAW + s), kCopy);
       mbar_init(BAR(BAR_KVE + s), 1);
       mbar_init(BAR(BAR_PF + s), 4);
     }
@@ -499,10 +572,11 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     mbar_init(BAR(BAR_FIN2), 1);
     mbar_init(BAR(BAR_QT), 4);
     mbar_init(BAR(BAR_QS), 1);
+    mbar_init(BAR(BAR_CS1), p.cluster ? p.nsplit : 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(BAR(BAR_IXF + r), 1);
       mbar_init(BAR(BAR_IXS + r), 1);
-      mbar_init(BAR(BAR_IXE + r), kLoad / 32 + 4);
+      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + 4);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -512,6 +586,9 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // Cluster launch: the barriers of every CTA are initialised before any
+  // CTA of the cluster can arrive on them remotely.
+  if (p.cluster) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kAuxTmem);
   SMLA_TRACE_EV(1);
@@ -586,29 +663,68 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       r1_0 = r2_0; r1_1 = r2_1;
       i2_0 = i3_0; i2_1 = i3_1;
     }
+  } else if (warp >= kWarpLoad0 + Cfg<kFp8>::kCopyWarps) {
+    // ------------------------------------------------- fp8 convert warps
+    // Thread (tok, sub) turns the 16 codes of dims [16 sub, 16 sub + 16) of
+    // every atom into bf16.  The copy warps put those codes in the first of
+    // the two 16-byte chunks their bf16 values occupy in the swizzled tile,
+    // so each thread reads and rewrites only its own two chunks: the
+    // conversion runs in place with no barrier between threads.
+    const int ct = threadIdx.x - 32 * (kWarpLoad0 + Cfg<kFp8>::kCopyWarps);  // 0 .. 255
+    const int tok = ct >> 2, sub = ct & 3;
+    for (int t = 0; t < ntiles; ++t) {
+      const int stage = t % kStages;
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + stage), (t / kStages) & 1))) break;
+      if (ct == 0 && t < 8) SMLA_TRACE_EV(40 + t);
+      const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
+#pragma unroll
+      for (int a = 0; a < kAtoms; ++a) {
+        const uint32_t lo_addr = tbase + a * kAtomBytes + sw128_off(tok, 2 * sub);
+        const uint4 v = ld_shared_v4(lo_addr);
+        uint4 lo, hi;
+        e4m3x4_to_bf16x4(v.x, lo.x, lo.y);
+        e4m3x4_to_bf16x4(v.y, lo.z, lo.w);
+        e4m3x4_to_bf16x4(v.z, hi.x, hi.y);
+        e4m3x4_to_bf16x4(v.w, hi.z, hi.w);
+        st_shared_v4(lo_addr, lo);
+        st_shared_v4(tbase + a * kAtomBytes + sw128_off(tok, 2 * sub + 1), hi);
+      }
+      // one proxy fence for the tile: generic stores -> tensor-core reads
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_KVF + stage));
+      if (ct == 0 && (t == 2 || t == 3)) SMLA_TRACE_EV(t == 2 ? 57 : 63);
+    }
   } else if (warp >= kWarpLoad0) {
-    // ------------------------------------------------------------ loaders
-    const int lt = threadIdx.x - 32 * kWarpLoad0;  // 0 .. kLoad-1
+    // ------------------------------------------------------- copy warps
+    const int lt = threadIdx.x - 32 * kWarpLoad0;  // 0 .. kCopy-1
+    const int lw = lt >> 5;
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages, rs = t % kRing;
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1))) break;  // warp-uniform
       const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
+      // bf16: lane covers tokens 4u + lane/8, 16-byte chunk lane%8 of a
+      // 128-byte atom row; fp8: tokens 8(4 lw + u) + lane/4, 16 codes
+      // (chunk lane%4) of a 64-byte atom row
+      int rows[16];
       if constexpr (!kFp8) {
-        // Loader warp w copies atoms w, w+4, w+8: 64 rows x 8 chunks of 16 B
-        // per atom, 16 per lane; each warp instruction covers four whole
-        // 128-byte row segments (coalesced).  Padding rows are zero-filled
-        // (source size 0).
-        const int lw = lt >> 5;
-        int rows[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) rows[u] = s_row[rs * 64 + 4 * u + (lane >> 3)];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
-          break;
-        // stage 2 first holds the staged query
-        if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) rows[u] = s_row[rs * 64 + 8 * (4 * lw + u) + (lane >> 2)];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
+      if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+        break;
+      // stage 2 first holds the staged query
+      if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
+      if constexpr (!kFp8) {
         if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
+        // warp w copies atoms w, w+4, w+8; each warp instruction covers four
+        // whole 128-byte row segments (coalesced); padding rows are
+        // zero-filled (source size 0)
         const int j = lane & 7;
 #pragma unroll 1
         for (int a = lw; a < kAtoms; a += 4) {
@@ -622,45 +738,23 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
       } else {
-        // thread (tok = lt/4, sub = lt%4): 16 codes of every atom; loads are
-        // issued before the stage is free and converted once it is
-        const int tok = lt >> 2, sub = lt & 3;
-        const int row = s_row[rs * 64 + tok];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-        uint4 v[kAtoms];
+        if (lt == 0 && t < 8) SMLA_TRACE_EV(48 + t);
+        // each warp instruction covers eight 64-byte row segments; codes go
+        // to the first chunk of their bf16 destination (see the convert warps)
+        const int sub = lane & 3;
 #pragma unroll
-        for (int a = 0; a < kAtoms; ++a)
-          v[a] = row >= 0 ? ld_global_nc_v4(p.kv + (size_t)row * kRowBytesFp8 + a * 64 + sub * 16)
-                          : make_uint4(0, 0, 0, 0);
-        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
-          break;
-        // stage 2 first holds the staged query
-        if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
-        if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
+        for (int u = 0; u < 4; ++u) {
+          const int tok = 8 * (4 * lw + u) + (lane >> 2);
+          const int row = rows[u];
+          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8 + sub * 16;
 #pragma unroll
-        for (int a = 0; a < kAtoms; ++a) {
-          uint4 lo, hi;
-          lo.x = e4m3x2_to_bf16x2((uint16_t)(v[a].x & 0xFFFF));
-          lo.y = e4m3x2_to_bf16x2((uint16_t)(v[a].x >> 16));
-          lo.z = e4m3x2_to_bf16x2((uint16_t)(v[a].y & 0xFFFF));
-          lo.w = e4m3x2_to_bf16x2((uint16_t)(v[a].y >> 16));
-          hi.x = e4m3x2_to_bf16x2((uint16_t)(v[a].z & 0xFFFF));
-          hi.y = e4m3x2_to_bf16x2((uint16_t)(v[a].z >> 16));
-          hi.z = e4m3x2_to_bf16x2((uint16_t)(v[a].w & 0xFFFF));
-          hi.w = e4m3x2_to_bf16x2((uint16_t)(v[a].w >> 16));
-          const uint32_t rb = tbase + a * kAtomBytes;
-          st_shared_v4(rb + sw128_off(tok, 2 * sub), lo);
-          st_shared_v4(rb + sw128_off(tok, 2 * sub + 1), hi);
+          for (int a = 0; a < kAtoms; ++a)
+            cp_async_16(tbase + a * kAtomBytes + sw128_off(tok, 2 * sub), src + a * 64, row >= 0 ? 16u : 0u);
         }
-        // one proxy fence for the whole tile: generic stores -> tensor-core reads
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_KVF + stage));
+        cp_async_mbar_arrive_noinc(BAR(BAR_RAW + stage));
       }
-      if (lt == 0 && t == 2) SMLA_TRACE_EV(57);
     }
-    if (!kFp8) cp_async_wait_all();
+    cp_async_wait_all();
   } else if (warp == kWarpS || warp == kWarpPV) {
     // ------------------------------------------------------------ MMA issuers
     // Two warps issue tensor-core work, each blocking (in hardware) on one
@@ -881,7 +975,131 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       tc_fence_after();
     }
     if (threadIdx.x == 0) SMLA_TRACE_EV(3);
-    if (!aborted) {
+    // the cluster reduction synchronises the four warps: enter it together
+    if (p.cluster) aborted = group_any(aborted, 1, 128);
+    if (!aborted && p.cluster) {
+      // ------------------------------------- split merge inside the cluster
+      // The nsplit CTAs of this sequence form a cluster (rank = split); the
+      // exchange goes through the workspace (L2), one launch in all.
+      // 1. Each CTA stores its O, unnormalised, straight from registers in
+      //    "register image" order (for warp w, chunk c, vector u: 32 lanes x
+      //    16 bytes contiguous, so every warp store covers 512 bytes), and
+      //    its per-head (m, l, l_pv).
+      // 2. One cluster-wide barrier: remote mbarrier arrivals (release),
+      //    bounded waits (acquire).
+      // 3. CTA r owns output columns [r cn, (r+1) cn), cn = 512 / nsplit.
+      //    Thread (head hh, part) reads its 256 / nsplit columns of every
+      //    split s (16 lanes x 16 bytes contiguous per load), weights them
+      //    by 2^(m_s - M), divides by the equally weighted sum of the
+      //    rounded-P sums (the normalisation of one CTA over all tiles) and
+      //    writes them; rank 0 writes lse.
+      const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
+      const int n = p.nsplit;
+      float4* wso = reinterpret_cast<float4*>(p.part_o) + (size_t)b * n * (kH * kDv / 4);   // [src][w][c][u][lane]
+      float* wss = p.part_lse + (size_t)b * n * 64 * 4;          // [src][64][4]: m, l, l_pv
+      {
+        float4* mine = wso + (size_t)split * (kH * kDv / 4) + (size_t)warp * (8 * 8 * 32) + lane;
+        // tensor-memory loads run one chunk ahead of the stores
+        float o[2][32];
+        if (ntiles > 0) {
+          tmem_ld_16x32bx2_x32_h256(tmem + o_lanes, o[0]);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) { o[0][k] = 0.f; o[1][k] = 0.f; }
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          if (ntiles > 0 && c + 1 < 8) tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)(c + 1), o[(c + 1) & 1]);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            mine[(c * 8 + u) * 32] = make_float4(o[c & 1][4 * u], o[c & 1][4 * u + 1], o[c & 1][4 * u + 2],
+                                                 o[c & 1][4 * u + 3]);
+          if (ntiles > 0 && c + 1 < 8) tmem_wait_ld();
+        }
+      }
+      if (half == 0) {
+        float4* st4 = reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4);
+        *st4 = make_float4(m_run, l_tot, l_nrm, 0.f);
+      }
+      named_bar_sync(1, 128);
+      if (threadIdx.x == 0) {
+        fence_acq_rel_cluster();
+        for (int r = 0; r < n; ++r) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)r));
+      }
+      if (threadIdx.x == 0) SMLA_TRACE_EV(4);
+      // every CTA of the cluster has written (and no CTA exits before this
+      // wait: the remote arrivals target live CTAs)
+      bool ok = mbar_wait_cluster(BAR(BAR_CS1), 0);
+      if (threadIdx.x == 0) SMLA_TRACE_EV(7);
+      if (group_any(!ok, 1, 128)) {
+        aborted = true;
+      } else {
+        // this thread: head hh = 16 w + lane % 16, which lives in lane
+        // hh % 16 (+16 for dims >= 256) of warp w of every split
+        const int hh = h, sub = half;
+        float mv[16];
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2)
+          if (s2 < n) mv[s2] = __ldcg(wss + ((size_t)s2 * 64 + hh) * 4);
+        float M = -INFINITY;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2)
+          if (s2 < n) M = fmaxf(M, mv[s2]);
+        float Lr = 0.f, Lp = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) {
+          if (s2 < n) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
+            const float wgt = mv[s2] > -INFINITY ? ex2(mv[s2] - M) : 0.f;
+            mv[s2] = wgt;                  // from here on: the weight of split s2
+            Lr += wgt * v.y;
+            Lp += wgt * v.z;
+          }
+        }
+        const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
+        if (split == 0 && sub == 0)
+          p.lse[(size_t)b * kH + hh] = Lr > 0.f ? (M + log2f(Lr)) * 0.6931471805599453f : -INFINITY;
+        if (threadIdx.x == 0) SMLA_TRACE_EV(56);
+        // this CTA's columns [split cn, +cn); this thread takes vectors
+        // [v0, v0 + nv) of them (4 columns each), nv = 64 / n
+        const int cn = kDv / n;
+        const int nv = cn / 8;
+        const int col0 = split * cn + sub * (cn / 2);            // first column of this thread
+        const int hf = col0 >> 8;                                // which lane half stores them
+        const float4* src = wso + (size_t)warp * (8 * 8 * 32) + (lane & 15) + 16 * hf;
+        __nv_bfloat16* orow = p.out + ((size_t)b * kH + hh) * kDv + col0;
+#pragma unroll 1
+        for (int v0 = 0; v0 < nv; v0 += 4) {
+          float4 a[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int s2 = 0; s2 < 16; ++s2) {
+            if (s2 < n) {
+              const float wgt = mv[s2];
+              const float4* ss = src + (size_t)s2 * (kH * kDv / 4);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int d = (col0 & 255) + 4 * (v0 + k);       // dim within the half, multiple of 4
+                const float4 v = __ldcg(ss + ((d >> 5) * 8 + ((d >> 2) & 7)) * 32);
+                a[k].x += wgt * v.x; a[k].y += wgt * v.y; a[k].z += wgt * v.z; a[k].w += wgt * v.w;
+              }
+            }
+          }
+          uint4 ov;
+          ov.x = pack_bf16x2(a[0].x * inv, a[0].y * inv); ov.y = pack_bf16x2(a[0].z * inv, a[0].w * inv);
+          ov.z = pack_bf16x2(a[1].x * inv, a[1].y * inv); ov.w = pack_bf16x2(a[1].z * inv, a[1].w * inv);
+          *reinterpret_cast<uint4*>(orow + 4 * v0) = ov;
+          ov.x = pack_bf16x2(a[2].x * inv, a[2].y * inv); ov.y = pack_bf16x2(a[2].z * inv, a[2].w * inv);
+          ov.z = pack_bf16x2(a[3].x * inv, a[3].y * inv); ov.w = pack_bf16x2(a[3].z * inv, a[3].w * inv);
+          *reinterpret_cast<uint4*>(orow + 4 * v0 + 8) = ov;
+        }
+        if (threadIdx.x == 0) SMLA_TRACE_EV(62);
+      }
+      if (threadIdx.x == 0) SMLA_TRACE_EV(5);
+    } else if (!aborted) {
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       const bool any = l_tot > 0.f;
@@ -1015,7 +1233,7 @@ static int device_sm_count() {
   return n;
 }
 
-static int plan_nsplit(const smla_shape* s, int num_sms) {
+static int plan_nsplit_raw(const smla_shape* s, int num_sms) {
   const int tiles = (s->topk + kTile - 1) / kTile;
   int n;
   if (s->nsplit > 0) {
@@ -1028,10 +1246,51 @@ static int plan_nsplit(const smla_shape* s, int num_sms) {
   return n;
 }
 
+// The split plan: n CTAs per sequence, each over a contiguous run of tiles.
+// cluster: the n CTAs form a thread-block cluster and merge inside the
+// split kernel (no combine kernel); possible when n is a power of two no
+// larger than 16 that the device can launch as a cluster.  An explicit
+// nsplit is kept as given (merged in the kernel whenever it can launch as a
+// cluster); an automatic plan takes the largest such n that fits in one
+// wave (falling back to one split).
+struct Plan {
+  int n;
+  bool cluster;
+};
+static Plan make_plan(const smla_shape* s, int num_sms, const int active[5]) {
+  Plan pl{plan_nsplit_raw(s, num_sms), false};
+  if (pl.n < 2) return pl;
+  if (s->nsplit > 0) {
+    if ((pl.n & (pl.n - 1)) == 0 && pl.n <= 16) pl.cluster = active[31 - __builtin_clz(pl.n)] >= 1;
+    return pl;
+  }
+  // The largest power-of-two split (<= the raw count) whose B clusters are
+  // all resident at once; on B200 this measured within a few percent of the
+  // best split count for every batch and list length tried.
+  for (int lg = 4; lg >= 1; --lg) {
+    const int c = 1 << lg;
+    if (c <= pl.n && active[lg] >= s->batch) return Plan{c, true};
+  }
+  return Plan{1, false};
+}
+
 static size_t partial_bytes(int batch, int nsplit) {
   const size_t o = (size_t)batch * nsplit * kH * kDv * 4;
   const size_t l = (size_t)batch * nsplit * kH * 4;
   return ((o + l + 255) / 256) * 256;
+}
+
+// Workspace of an in-cluster merge: every CTA's O as nsplit column blocks
+// (B * nsplit * 64 * 512 fp32) and its per-head (m, l, l_pv, -) (B * nsplit
+// * 64 * 4 fp32).
+static size_t cluster_bytes(int batch, int nsplit) {
+  const size_t o = (size_t)batch * nsplit * kH * kDv * 4;
+  const size_t st = (size_t)batch * nsplit * kH * 4 * 4;
+  return ((o + st + 255) / 256) * 256;
+}
+static size_t workspace_bytes_for(int batch, int nsplit, bool cluster) {
+  if (nsplit < 2) return 0;
+  return cluster ? cluster_bytes(batch, nsplit) : partial_bytes(batch, nsplit);
 }
 
 // The shared-memory opt-in is set once per device (an idempotent call, so a
@@ -1049,20 +1308,79 @@ static cudaError_t ensure_smem_attr() {
   return e;
 }
 
+// How many clusters of c split CTAs (c = 2, 4, 8, 16) the device holds at
+// once for this kernel (1 CTA per SM: a cluster needs c SMs of one GPC).
+// Queried once per device; 0 = that size cannot launch.
+struct ClusterCaps {
+  int active[5];  // index log2(c); active[0] unused
+};
+template <bool kFp8>
+static const ClusterCaps& cluster_caps() {
+  static ClusterCaps cache[64];
+  static volatile int done[64] = {0};
+  static ClusterCaps none = {{0, 0, 0, 0, 0}};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return none;
+  if (done[dev]) return cache[dev];
+  ClusterCaps caps = {{0, 0, 0, 0, 0}};
+  if (ensure_smem_attr<kFp8>() == cudaSuccess &&
+      cudaFuncSetAttribute(smla_split_kernel<kFp8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+          cudaSuccess) {
+    for (int lg = 1; lg <= 4; ++lg) {
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 1u << lg;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1u << lg, 1, 1);
+      cfg.blockDim = dim3(Cfg<kFp8>::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kSmemBytes;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int k = 0;
+      if (cudaOccupancyMaxActiveClusters(&k, smla_split_kernel<kFp8>, &cfg) == cudaSuccess) caps.active[lg] = k;
+    }
+  }
+  cudaGetLastError();  // a refused query leaves no sticky error
+  cache[dev] = caps;
+  done[dev] = 1;
+  return cache[dev];
+}
+static const ClusterCaps& caps_for(const smla_shape* s) {
+  return s->kv_dtype == SMLA_KV_FP8_E4M3_ROWSCALE ? cluster_caps<true>() : cluster_caps<false>();
+}
+
 template <bool kFp8>
 static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
   auto kern = smla_split_kernel<kFp8>;
   cudaError_t e = ensure_smem_attr<kFp8>();
   if (e != cudaSuccess) return e;
   dim3 grid(prm.nsplit, prm.batch);
-  kern<<<grid, Cfg<kFp8>::kThreads, kSmemBytes, stream>>>(prm);
-  return cudaGetLastError();
+  if (!prm.cluster) {
+    kern<<<grid, Cfg<kFp8>::kThreads, kSmemBytes, stream>>>(prm);
+    return cudaGetLastError();
+  }
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = prm.nsplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(Cfg<kFp8>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
 static smla_status run_split(const smla_shape* shape, const void* q, const void* kv_cache,
                              const float* kv_row_scale, const int32_t* page_table, const int32_t* indices,
                              float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                             int32_t* nsplit_out, cudaStream_t stream, int* nsplit_used) {
+                             int32_t* nsplit_out, cudaStream_t stream, int* nsplit_used, bool allow_cluster,
+                             bool* cluster_used) {
   smla_status st = validate_shape(shape);
   if (st != SMLA_OK) return st;
   if (!q || !kv_cache || !indices || !out || !lse) return SMLA_ERR_INVALID_ARG;
@@ -1074,10 +1392,12 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   if (!(scale == scale) || isinf(scale)) return SMLA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   if (sms <= 0) return SMLA_ERR_CUDA;
-  const int n = plan_nsplit(shape, sms);
+  const Plan pl = make_plan(shape, sms, caps_for(shape).active);
+  const int n = pl.n;
+  const bool cluster = allow_cluster && pl.cluster;
   if (n > 1) {
     if (!workspace || !aligned(workspace, 256)) return SMLA_ERR_WORKSPACE;
-    if (workspace_bytes < partial_bytes(shape->batch, n)) return SMLA_ERR_WORKSPACE;
+    if (workspace_bytes < workspace_bytes_for(shape->batch, n, cluster)) return SMLA_ERR_WORKSPACE;
   }
   SplitParams prm;
   memset(&prm, 0, sizeof(prm));
@@ -1088,6 +1408,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.indices = indices;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
+  prm.cluster = cluster ? 1 : 0;
   prm.part_o = static_cast<float*>(workspace);
   prm.part_lse = n > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
                                                   (size_t)shape->batch * n * kH * kDv * 4)
@@ -1103,6 +1424,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   if (e != cudaSuccess) return SMLA_ERR_CUDA;
   if (nsplit_out) *nsplit_out = n;
   if (nsplit_used) *nsplit_used = n;
+  if (cluster_used) *cluster_used = cluster;
   return SMLA_OK;
 }
 
@@ -1151,13 +1473,19 @@ const char* sparse_mla_status_string(smla_status s) {
 
 int32_t sparse_mla_plan_nsplit(const smla_shape* shape) {
   if (smla::validate_shape(shape) != SMLA_OK) return 0;
-  return smla::plan_nsplit(shape, smla::device_sm_count());
+  return smla::make_plan(shape, smla::device_sm_count(), smla::caps_for(shape).active).n;
 }
 
 size_t sparse_mla_workspace_size(const smla_shape* shape) {
   if (smla::validate_shape(shape) != SMLA_OK) return 0;
-  const int n = smla::plan_nsplit(shape, smla::device_sm_count());
-  return n > 1 ? smla::partial_bytes(shape->batch, n) : 0;
+  const smla::Plan pl = smla::make_plan(shape, smla::device_sm_count(), smla::caps_for(shape).active);
+  return smla::workspace_bytes_for(shape->batch, pl.n, pl.cluster);
+}
+
+int32_t sparse_mla_plan_merge(const smla_shape* shape) {
+  if (smla::validate_shape(shape) != SMLA_OK) return -1;
+  const smla::Plan pl = smla::make_plan(shape, smla::device_sm_count(), smla::caps_for(shape).active);
+  return pl.n < 2 ? 0 : (pl.cluster ? 1 : 2);
 }
 
 smla_status sparse_mla_decode_split(const smla_shape* shape, const void* q, const void* kv_cache,
@@ -1166,7 +1494,7 @@ smla_status sparse_mla_decode_split(const smla_shape* shape, const void* q, cons
                                     void* workspace, size_t workspace_bytes, int32_t* nsplit_out,
                                     void* stream) {
   return smla::run_split(shape, q, kv_cache, kv_row_scale, page_table, indices, scale, out, lse, workspace,
-                         workspace_bytes, nsplit_out, static_cast<cudaStream_t>(stream), nullptr);
+                         workspace_bytes, nsplit_out, static_cast<cudaStream_t>(stream), nullptr, false, nullptr);
 }
 
 smla_status sparse_mla_decode(const smla_shape* shape, const void* q, const void* kv_cache,
@@ -1174,10 +1502,11 @@ smla_status sparse_mla_decode(const smla_shape* shape, const void* q, const void
                               float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                               void* stream) {
   int n = 0;
+  bool cluster = false;
   const smla_status st = smla::run_split(shape, q, kv_cache, kv_row_scale, page_table, indices, scale, out, lse,
                                          workspace, workspace_bytes, nullptr, static_cast<cudaStream_t>(stream),
-                                         &n);
-  if (st != SMLA_OK || n == 1) return st;
+                                         &n, true, &cluster);
+  if (st != SMLA_OK || n == 1 || cluster) return st;
   const float* po = static_cast<const float*>(workspace);
   const float* pl = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) +
                                                    (size_t)shape->batch * n * smla::kH * smla::kDv * 4);
@@ -1202,10 +1531,17 @@ smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void
                                              void* stream) {
   smla_status st = smla::validate_shape(shape);
   if (st != SMLA_OK) return st;
-  // split count and scratch need: no CUDA call when the caller fixes nsplit
-  const int n = shape->nsplit > 0 ? smla::plan_nsplit(shape, 0) : smla::plan_nsplit(shape, smla::device_sm_count());
-  if (shape->nsplit == 0 && smla::device_sm_count() <= 0) return SMLA_ERR_CUDA;
-  const size_t need = n > 1 ? smla::partial_bytes(shape->batch, n) : 0;
+  // split count and scratch need (no CUDA call when the caller fixes an
+  // nsplit whose partials cannot fit, whichever way they are merged)
+  if (shape->nsplit > 0) {
+    const int n0 = smla::plan_nsplit_raw(shape, 0);
+    if (n0 > 1 && smla::partial_bytes(shape->batch, n0) > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
+  }
+  const int sms = smla::device_sm_count();
+  if (sms <= 0) return SMLA_ERR_CUDA;
+  const smla::Plan pl = smla::make_plan(shape, sms, smla::caps_for(shape).active);
+  const int n = pl.n;
+  const size_t need = smla::workspace_bytes_for(shape->batch, n, pl.cluster);
   if (need > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (need > 0) {

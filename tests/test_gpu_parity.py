@@ -138,6 +138,73 @@ def test_single_index_is_bit_exact_value_row():
     np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-5, atol=1e-5)
 
 
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("n", [2, 4, 8, 16])
+def test_cluster_merge_every_size(n, fp8):
+    """nsplit a power of two no larger than the cluster limit: the CTAs of a
+    sequence merge their splits inside the split kernel.  Oracle parity,
+    including a sequence whose later splits hold only padding (weight 0) and
+    an all-padding sequence (out 0, lse -inf)."""
+    if fp8:
+        w = inputs.paged_fp8(3, 4096, 256, 2048, seed=60 + n)
+    else:
+        w = inputs.flat_per_seq(3, 8192, 2048, seed=40 + n)
+    w.indices[1, 700:] = -1
+    w.indices[2] = -1
+    d = Dev(w)
+    a = api()
+    shape = a.shape_for(d.q, d.kv, d.indices, page_table=d.page_table, page_size=w.page_size, nsplit=n)
+    assert a.plan_nsplit(shape) == n
+    if n <= 8:                      # portable cluster sizes always launch
+        assert a.plan_merge(shape) == 1
+    out, lse = d.run(nsplit=n)
+    torch.cuda.synchronize()
+    out_ref, lse_ref = oracle(w, seqs=[0, 1])
+    assert_parity(out, lse, out_ref, lse_ref, seqs=[0, 1], tag=f"cluster n={n}")
+    assert torch.all(out[2].float() == 0) and torch.all(torch.isneginf(lse[2]))
+
+
+def test_cluster_merge_counting_exact():
+    """On-chip merge over 8 splits recovers the exact set of gathered rows."""
+    w, weights, nval = counting_workload(3, 2048, 8192, fp8=False, paged=False, seed=77)
+    d = Dev(w)
+    out, lse = d.run(nsplit=8)
+    torch.cuda.synchronize()
+    o = out.float().cpu().numpy().astype(np.float64)
+    for b in range(3):
+        got = np.rint(o[b] * nval[b] * 2) / 2
+        assert np.array_equal(got, np.broadcast_to(weights[b], got.shape)), f"seq {b}"
+        np.testing.assert_allclose(lse[b].cpu().numpy(), np.log(nval[b]), rtol=1e-6)
+
+
+def test_fp8_every_code_decodes_exactly():
+    """One index per sequence gives out = the gathered value row, so every
+    non-NaN e4m3fn code, times a power-of-two row scale, must come back as
+    its exact bf16 value (subnormal codes included).  Values are compared,
+    so -0 equals +0: the weighted sum over a tile adds +0 from the padding
+    rows, which turns the code -0 into +0."""
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    N = 16
+    kv = np.stack([codes[(np.arange(576) + 37 * r) % codes.size] for r in range(N)])
+    scales = np.array([2.0 ** ((r % 7) - 3) for r in range(N)], dtype=np.float32)
+    idx = np.array([[2], [7], [11], [13]], dtype=np.int32)
+    q = inputs._normal_bf16(torch.Generator().manual_seed(21), (4, 64, 576))
+    w = inputs.Workload(name="fp8_codes", q=q, kv=torch.from_numpy(kv), indices=torch.from_numpy(idx),
+                        kv_row_scale=torch.from_numpy(scales))
+    d = Dev(w)
+    out, lse = d.run()
+    torch.cuda.synchronize()
+    for b in range(4):
+        r = int(idx[b, 0])
+        vals = ref.e4m3fn_to_f64(kv[r, :512]) * float(scales[r])    # exact in bf16
+        got = out[b].float().cpu().numpy().astype(np.float64)
+        assert np.array_equal(got, np.broadcast_to(vals, got.shape)), f"row {r}"
+    # lse = the one score, an fp32 sum of 576 products of magnitude up to
+    # 448 |q| (rounding ~1e-3 absolute): the parity gate
+    _, lse_ref = oracle(w)
+    assert np.max(ref.lse_rel_err(lse.cpu().numpy(), lse_ref)) <= 1e-3
+
+
 def test_all_padding_sequence_and_mixed():
     w = inputs.flat_per_seq(3, 800, 130, seed=4)
     w.indices[1] = -1
@@ -245,7 +312,7 @@ def test_deterministic_bits():
     assert torch.equal(a[0].view(torch.int16), b[0].view(torch.int16)) and torch.equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("name", ["c1", "c3"])
+@pytest.mark.parametrize("name", ["c1", "c3", "c4a"])     # c4a: the in-cluster merge
 def test_cuda_graph_replay_bit_identical(name):
     w = inputs.make_config(name)
     d = Dev(w)

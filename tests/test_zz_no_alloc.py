@@ -25,7 +25,7 @@ def _static(shape, q=16, kv=16, idx=16, out=16, lse=16):
                                                     out, lse, None)
 
 
-@pytest.mark.parametrize("batch,topk,nsplit", [(64, 512, 8), (96, 128, 2), (1, 2048 * 64, 200)])
+@pytest.mark.parametrize("batch,topk,nsplit", [(64, 512, 6), (64, 192, 3), (1, 2048 * 64, 200)])
 def test_over_the_limit_rejected_before_any_cuda_call(batch, topk, nsplit):
     assert batch * nsplit * PARTIAL_BYTES > api.STATIC_SCRATCH_BYTES
     s = api.make_shape(batch, topk, 100000, nsplit=nsplit)
@@ -38,8 +38,9 @@ def test_limit_constant_matches_header():
     hdr = open(os.path.join(os.path.dirname(api.__file__), "..", "include", "sparse_mla.h")).read()
     m = re.search(r"#define SMLA_STATIC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
     assert m and int(m.group(1)) << int(m.group(2)) == api.STATIC_SCRATCH_BYTES
-    # every split count the planner picks on a 148-SM part fits
-    assert 148 * PARTIAL_BYTES <= api.STATIC_SCRATCH_BYTES
+    # every split count the planner picks on a 148-SM part fits, merged
+    # either way (in-cluster merges keep 64 x 4 floats of statistics)
+    assert 148 * (PARTIAL_BYTES - 64 * 4 + 64 * 16) <= api.STATIC_SCRATCH_BYTES
 
 
 def _dev(w):
@@ -52,6 +53,7 @@ def _dev(w):
 CASES = {
     "varlen_planned": (lambda: inputs.flat_varlen(4, 100, 900, 512, seed=77), 0),
     "flat_nsplit5": (lambda: inputs.flat_per_seq(2, 2048, 700, seed=78), 5),
+    "flat_nsplit4_on_chip": (lambda: inputs.flat_per_seq(2, 2048, 700, seed=82), 4),
     "paged_fp8_planned": (lambda: inputs.paged_fp8(3, 1024, 64, 300, seed=79), 0),
     "single_split": (lambda: inputs.flat_per_seq(2, 1024, 200, seed=80), 1),
 }
@@ -79,21 +81,22 @@ def test_two_calls_in_a_row_match_sparse_mla_decode(case):
 
 @pytest.mark.gpu
 def test_largest_fitting_and_first_rejected_shape_on_gpu():
-    # 95 x 2 partials fit in the scratch, 96 x 2 do not
-    assert 95 * 2 * PARTIAL_BYTES <= api.STATIC_SCRATCH_BYTES < 96 * 2 * PARTIAL_BYTES
-    w = inputs.flat_per_seq(96, 256, 128, seed=81)
+    # 63 x 3 partials fit in the scratch, 64 x 3 do not (3 splits merge
+    # through partials: not a power of two)
+    assert 63 * 3 * PARTIAL_BYTES <= api.STATIC_SCRATCH_BYTES < 64 * 3 * PARTIAL_BYTES
+    w = inputs.flat_per_seq(64, 256, 192, seed=81)
     t = _dev(w)
-    q95, i95 = t["q"][:95].contiguous(), t["indices"][:95].contiguous()
-    want_o, want_l = api.decode(q95, t["kv"], i95, w.scale, nsplit=2)
-    out = torch.empty((95, 64, 512), dtype=torch.bfloat16, device="cuda")
-    lse = torch.empty((95, 64), dtype=torch.float32, device="cuda")
-    api.decode_static_scratch(q95, t["kv"], i95, w.scale, out, lse, nsplit=2)
+    q63, i63 = t["q"][:63].contiguous(), t["indices"][:63].contiguous()
+    want_o, want_l = api.decode(q63, t["kv"], i63, w.scale, nsplit=3)
+    out = torch.empty((63, 64, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((63, 64), dtype=torch.float32, device="cuda")
+    api.decode_static_scratch(q63, t["kv"], i63, w.scale, out, lse, nsplit=3)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), want_o.view(torch.int16))
     assert torch.equal(lse.view(torch.int32), want_l.view(torch.int32))
-    out96 = torch.empty((96, 64, 512), dtype=torch.bfloat16, device="cuda")
-    lse96 = torch.empty((96, 64), dtype=torch.float32, device="cuda")
+    out64 = torch.empty((64, 64, 512), dtype=torch.bfloat16, device="cuda")
+    lse64 = torch.empty((64, 64), dtype=torch.float32, device="cuda")
     with pytest.raises(api.SmlaError) as e:
-        api.decode_static_scratch(t["q"], t["kv"], t["indices"], w.scale, out96, lse96, nsplit=2)
+        api.decode_static_scratch(t["q"], t["kv"], t["indices"], w.scale, out64, lse64, nsplit=3)
     assert e.value.code == WORKSPACE
     assert api.device_error() == 0
