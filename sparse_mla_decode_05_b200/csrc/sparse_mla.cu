@@ -593,6 +593,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kAuxTmem);
   SMLA_TRACE_EV(1);
 
+  bool merge_failed = false;   // a softmax warp gave up (in-cluster merge)
   if (warp >= kWarpIdx && warp < kWarpIdx + kIdxWarps) {
     // ------------------------------------------------------------ index warps
     // Resolve each tile's 64 entries to physical rows (and fp8 row scales)
@@ -677,17 +678,20 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + stage), (t / kStages) & 1))) break;
       if (ct == 0 && t < 8) SMLA_TRACE_EV(40 + t);
       const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
+      const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
+      // all nine loads first (independent), then convert and store
+      uint4 v[kAtoms];
+#pragma unroll
+      for (int a = 0; a < kAtoms; ++a) v[a] = ld_shared_v4(tbase + a * kAtomBytes + lo_off);
 #pragma unroll
       for (int a = 0; a < kAtoms; ++a) {
-        const uint32_t lo_addr = tbase + a * kAtomBytes + sw128_off(tok, 2 * sub);
-        const uint4 v = ld_shared_v4(lo_addr);
         uint4 lo, hi;
-        e4m3x4_to_bf16x4(v.x, lo.x, lo.y);
-        e4m3x4_to_bf16x4(v.y, lo.z, lo.w);
-        e4m3x4_to_bf16x4(v.z, hi.x, hi.y);
-        e4m3x4_to_bf16x4(v.w, hi.z, hi.w);
-        st_shared_v4(lo_addr, lo);
-        st_shared_v4(tbase + a * kAtomBytes + sw128_off(tok, 2 * sub + 1), hi);
+        e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
+        e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
+        e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
+        e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
+        st_shared_v4(tbase + a * kAtomBytes + lo_off, lo);
+        st_shared_v4(tbase + a * kAtomBytes + hi_off, hi);
       }
       // one proxy fence for the tile: generic stores -> tensor-core reads
       fence_proxy_async_smem();
@@ -975,130 +979,16 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       tc_fence_after();
     }
     if (threadIdx.x == 0) SMLA_TRACE_EV(3);
-    // the cluster reduction synchronises the four warps: enter it together
-    if (p.cluster) aborted = group_any(aborted, 1, 128);
-    if (!aborted && p.cluster) {
-      // ------------------------------------- split merge inside the cluster
-      // The nsplit CTAs of this sequence form a cluster (rank = split); the
-      // exchange goes through the workspace (L2), one launch in all.
-      // 1. Each CTA stores its O, unnormalised, straight from registers in
-      //    "register image" order (for warp w, chunk c, vector u: 32 lanes x
-      //    16 bytes contiguous, so every warp store covers 512 bytes), and
-      //    its per-head (m, l, l_pv).
-      // 2. One cluster-wide barrier: remote mbarrier arrivals (release),
-      //    bounded waits (acquire).
-      // 3. CTA r owns output columns [r cn, (r+1) cn), cn = 512 / nsplit.
-      //    Thread (head hh, part) reads its 256 / nsplit columns of every
-      //    split s (16 lanes x 16 bytes contiguous per load), weights them
-      //    by 2^(m_s - M), divides by the equally weighted sum of the
-      //    rounded-P sums (the normalisation of one CTA over all tiles) and
-      //    writes them; rank 0 writes lse.
+    if (p.cluster) {
+      // in-cluster merge (after the warp roles): this split's per-head
+      // statistics (max, fp32 sum, rounded-P sum) go to the workspace
+      merge_failed = aborted;
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
-      const int n = p.nsplit;
-      float4* wso = reinterpret_cast<float4*>(p.part_o) + (size_t)b * n * (kH * kDv / 4);   // [src][w][c][u][lane]
-      float* wss = p.part_lse + (size_t)b * n * 64 * 4;          // [src][64][4]: m, l, l_pv
-      {
-        float4* mine = wso + (size_t)split * (kH * kDv / 4) + (size_t)warp * (8 * 8 * 32) + lane;
-        // tensor-memory loads run one chunk ahead of the stores
-        float o[2][32];
-        if (ntiles > 0) {
-          tmem_ld_16x32bx2_x32_h256(tmem + o_lanes, o[0]);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) { o[0][k] = 0.f; o[1][k] = 0.f; }
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          if (ntiles > 0 && c + 1 < 8) tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)(c + 1), o[(c + 1) & 1]);
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            mine[(c * 8 + u) * 32] = make_float4(o[c & 1][4 * u], o[c & 1][4 * u + 1], o[c & 1][4 * u + 2],
-                                                 o[c & 1][4 * u + 3]);
-          if (ntiles > 0 && c + 1 < 8) tmem_wait_ld();
-        }
+      if (!aborted && half == 0) {
+        float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
+        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4) = make_float4(m_run, l_tot, l_nrm, 0.f);
       }
-      if (half == 0) {
-        float4* st4 = reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4);
-        *st4 = make_float4(m_run, l_tot, l_nrm, 0.f);
-      }
-      named_bar_sync(1, 128);
-      if (threadIdx.x == 0) {
-        fence_acq_rel_cluster();
-        for (int r = 0; r < n; ++r) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)r));
-      }
-      if (threadIdx.x == 0) SMLA_TRACE_EV(4);
-      // every CTA of the cluster has written (and no CTA exits before this
-      // wait: the remote arrivals target live CTAs)
-      bool ok = mbar_wait_cluster(BAR(BAR_CS1), 0);
-      if (threadIdx.x == 0) SMLA_TRACE_EV(7);
-      if (group_any(!ok, 1, 128)) {
-        aborted = true;
-      } else {
-        // this thread: head hh = 16 w + lane % 16, which lives in lane
-        // hh % 16 (+16 for dims >= 256) of warp w of every split
-        const int hh = h, sub = half;
-        float mv[16];
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2)
-          if (s2 < n) mv[s2] = __ldcg(wss + ((size_t)s2 * 64 + hh) * 4);
-        float M = -INFINITY;
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2)
-          if (s2 < n) M = fmaxf(M, mv[s2]);
-        float Lr = 0.f, Lp = 0.f;
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) {
-          if (s2 < n) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
-            const float wgt = mv[s2] > -INFINITY ? ex2(mv[s2] - M) : 0.f;
-            mv[s2] = wgt;                  // from here on: the weight of split s2
-            Lr += wgt * v.y;
-            Lp += wgt * v.z;
-          }
-        }
-        const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
-        if (split == 0 && sub == 0)
-          p.lse[(size_t)b * kH + hh] = Lr > 0.f ? (M + log2f(Lr)) * 0.6931471805599453f : -INFINITY;
-        if (threadIdx.x == 0) SMLA_TRACE_EV(56);
-        // this CTA's columns [split cn, +cn); this thread takes vectors
-        // [v0, v0 + nv) of them (4 columns each), nv = 64 / n
-        const int cn = kDv / n;
-        const int nv = cn / 8;
-        const int col0 = split * cn + sub * (cn / 2);            // first column of this thread
-        const int hf = col0 >> 8;                                // which lane half stores them
-        const float4* src = wso + (size_t)warp * (8 * 8 * 32) + (lane & 15) + 16 * hf;
-        __nv_bfloat16* orow = p.out + ((size_t)b * kH + hh) * kDv + col0;
-#pragma unroll 1
-        for (int v0 = 0; v0 < nv; v0 += 4) {
-          float4 a[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-          for (int s2 = 0; s2 < 16; ++s2) {
-            if (s2 < n) {
-              const float wgt = mv[s2];
-              const float4* ss = src + (size_t)s2 * (kH * kDv / 4);
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int d = (col0 & 255) + 4 * (v0 + k);       // dim within the half, multiple of 4
-                const float4 v = __ldcg(ss + ((d >> 5) * 8 + ((d >> 2) & 7)) * 32);
-                a[k].x += wgt * v.x; a[k].y += wgt * v.y; a[k].z += wgt * v.z; a[k].w += wgt * v.w;
-              }
-            }
-          }
-          uint4 ov;
-          ov.x = pack_bf16x2(a[0].x * inv, a[0].y * inv); ov.y = pack_bf16x2(a[0].z * inv, a[0].w * inv);
-          ov.z = pack_bf16x2(a[1].x * inv, a[1].y * inv); ov.w = pack_bf16x2(a[1].z * inv, a[1].w * inv);
-          *reinterpret_cast<uint4*>(orow + 4 * v0) = ov;
-          ov.x = pack_bf16x2(a[2].x * inv, a[2].y * inv); ov.y = pack_bf16x2(a[2].z * inv, a[2].w * inv);
-          ov.z = pack_bf16x2(a[3].x * inv, a[3].y * inv); ov.w = pack_bf16x2(a[3].z * inv, a[3].w * inv);
-          *reinterpret_cast<uint4*>(orow + 4 * v0 + 8) = ov;
-        }
-        if (threadIdx.x == 0) SMLA_TRACE_EV(62);
-      }
-      if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     } else if (!aborted) {
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
@@ -1155,6 +1045,130 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       }
       if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     }
+    tc_fence_before();
+  }
+
+  if (p.cluster && warp < 8) {
+    // ------------------------------------- split merge inside the cluster
+    // The nsplit CTAs of this sequence form a cluster (rank = split); the
+    // exchange goes through the workspace (L2), one launch in all, and
+    // warps 0-7 (the softmax warps and, their roles done, warps 4-7, which
+    // reach the same tensor-memory lanes: warp w and w + 4 share quarter w)
+    // share the work.
+    // 1. Each CTA stores its O, unnormalised, straight from tensor memory in
+    //    "register image" order ([quarter][chunk][vector][lane], so each
+    //    warp store covers 512 contiguous bytes); warps 0-3 take chunks
+    //    0-3, warps 4-7 chunks 4-7.  The softmax warps stored the per-head
+    //    (m, l, l_pv) already.
+    // 2. One cluster-wide barrier: remote mbarrier arrivals (release),
+    //    bounded waits (acquire).  Every CTA arrives and waits even after an
+    //    error, so no remote arrival targets a CTA that has exited.
+    // 3. CTA r owns output columns [r cn, (r+1) cn), cn = 512 / nsplit.
+    //    Thread (head hh, part 0-3) reads its cn / 4 columns of every split
+    //    (16 lanes x 16 contiguous bytes per load), weights split s by
+    //    2^(m_s - M), divides by the equally weighted sum of the rounded-P
+    //    sums (the normalisation of one CTA over all tiles) and writes bf16;
+    //    rank 0 writes lse.
+    const int n = p.nsplit;
+    const int q = warp & 3;                                  // tensor-memory lane quarter
+    const int upper = warp >> 2;                             // 0: softmax warp, 1: helper warp
+    constexpr size_t kSplit4 = (size_t)kH * kDv / 4;         // float4 per split
+    float4* wso = reinterpret_cast<float4*>(p.part_o) + (size_t)b * n * kSplit4;   // [src][q][c][u][lane]
+    const float* wss = p.part_lse + (size_t)b * n * 64 * 4;  // [src][64][4]: m, l, l_pv
+    bool failed = merge_failed;
+    if (upper) {
+      // every PV has completed (the PV issuer's drain barrier: one phase)
+      failed = !mbar_wait(BAR(BAR_FIN2), 0);
+      tc_fence_after();
+    }
+    const bool bad = group_any(failed, 1, 256);
+    if (!bad) {
+      float4* mine = wso + (size_t)split * kSplit4 + (size_t)q * (8 * 8 * 32) + lane;
+      const uint32_t olanes = (uint32_t)(32 * q + kLaneO) << 16;
+      float o[2][32];
+      const int c0 = 4 * upper;
+      if (ntiles > 0) {
+        tmem_ld_16x32bx2_x32_h256(tmem + olanes + 32u * (uint32_t)c0, o[0]);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) { o[0][k] = 0.f; o[1][k] = 0.f; }
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = c0 + cc;
+        if (ntiles > 0 && cc + 1 < 4) tmem_ld_16x32bx2_x32_h256(tmem + olanes + 32u * (uint32_t)(c + 1), o[(cc + 1) & 1]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          mine[(c * 8 + u) * 32] = make_float4(o[cc & 1][4 * u], o[cc & 1][4 * u + 1], o[cc & 1][4 * u + 2],
+                                               o[cc & 1][4 * u + 3]);
+        if (ntiles > 0 && cc + 1 < 4) tmem_wait_ld();
+      }
+    }
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0) {
+      fence_acq_rel_cluster();
+      for (int r = 0; r < n; ++r) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)r));
+    }
+    if (threadIdx.x == 0) SMLA_TRACE_EV(4);
+    const bool ok = mbar_wait_cluster(BAR(BAR_CS1), 0);
+    if (threadIdx.x == 0) SMLA_TRACE_EV(7);
+    if (!group_any(bad || !ok, 1, 256)) {
+      const int hh = 16 * q + (lane & 15);
+      const int part = (lane >> 4) + 2 * upper;
+      float mv[16];
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2)
+        if (s2 < n) mv[s2] = __ldcg(wss + ((size_t)s2 * 64 + hh) * 4);
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2)
+        if (s2 < n) M = fmaxf(M, mv[s2]);
+      float Lr = 0.f, Lp = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        if (s2 < n) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
+          const float wgt = mv[s2] > -INFINITY ? ex2(mv[s2] - M) : 0.f;
+          mv[s2] = wgt;                    // from here on: the weight of split s2
+          Lr += wgt * v.y;
+          Lp += wgt * v.z;
+        }
+      }
+      const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
+      if (split == 0 && part == 0)
+        p.lse[(size_t)b * kH + hh] = Lr > 0.f ? (M + log2f(Lr)) * 0.6931471805599453f : -INFINITY;
+      if (threadIdx.x == 0) SMLA_TRACE_EV(56);
+      // this thread: columns [col0, col0 + cn / 4), stored by lane
+      // hh % 16 (+16 for dims >= 256) of quarter q of every split
+      const int cn = kDv / n;
+      const int nv = cn / 16;                                  // float4 per thread (>= 2)
+      const int col0 = split * cn + part * (cn / 4);
+      const int hf = col0 >> 8;
+      const float4* src = wso + (size_t)q * (8 * 8 * 32) + (lane & 15) + 16 * hf;
+      __nv_bfloat16* orow = p.out + ((size_t)b * kH + hh) * kDv + col0;
+#pragma unroll 1
+      for (int v0 = 0; v0 < nv; v0 += 2) {
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) {
+          if (s2 < n) {
+            const float wgt = mv[s2];
+            const float4* ss = src + (size_t)s2 * kSplit4;
+            const int d = (col0 & 255) + 4 * v0;              // dim within the half, multiple of 8
+            const float4 x = __ldcg(ss + ((d >> 5) * 8 + ((d >> 2) & 7)) * 32);
+            const float4 y = __ldcg(ss + (((d + 4) >> 5) * 8 + (((d + 4) >> 2) & 7)) * 32);
+            a0.x += wgt * x.x; a0.y += wgt * x.y; a0.z += wgt * x.z; a0.w += wgt * x.w;
+            a1.x += wgt * y.x; a1.y += wgt * y.y; a1.z += wgt * y.z; a1.w += wgt * y.w;
+          }
+        }
+        *reinterpret_cast<uint4*>(orow + 4 * v0) =
+            make_uint4(pack_bf16x2(a0.x * inv, a0.y * inv), pack_bf16x2(a0.z * inv, a0.w * inv),
+                       pack_bf16x2(a1.x * inv, a1.y * inv), pack_bf16x2(a1.z * inv, a1.w * inv));
+      }
+      if (threadIdx.x == 0) SMLA_TRACE_EV(62);
+    }
+    if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     tc_fence_before();
   }
 
