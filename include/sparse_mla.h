@@ -184,7 +184,7 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
 /* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:
- * 24 MiB, enough for batch * nsplit <= 190 split results (at most 132,096
+ * 24 MiB, enough for batch * nsplit <= 191 split results (at most 131,328
  * bytes each).  Every split count the planner picks on a 148-SM B200 fits
  * (it keeps batch * nsplit <= 148). */
 #define SMLA_STATIC_SCRATCH_BYTES ((size_t)24 << 20)

@@ -44,6 +44,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 #include <math.h>
 #include <string.h>
@@ -262,6 +263,12 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+// two fp32 -> packed f16x2 (lo in the low half), round to nearest even
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 // two fp32 -> packed bf16x2 (lo in the low half), round to nearest even
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -519,6 +526,44 @@ __device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, u
 }
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// In-cluster merge, final step for one thread: columns [d0, d0 + 64 / N * 4)
+// of one head (d0 = dim within its 256-dim half) from the N splits' fp16
+// images at src (one 16-byte unit = 8 dims; unit u of the half lives at
+// ((u / 4) * 4 + u % 4) * 32 lanes), weighted by w[s], times inv, to bf16.
+template <int N>
+__device__ __forceinline__ void merge_columns(const uint4* src, int d0, const float* w, float inv,
+                                              __nv_bfloat16* orow) {
+  constexpr int kU = 16 / N;                     // units per split (16 loads in all)
+  constexpr size_t kSplitU = (size_t)kH * kDv / 8;
+  uint4 x[16];
+#pragma unroll
+  for (int s = 0; s < N; ++s)
+#pragma unroll
+    for (int k = 0; k < kU; ++k) {
+      const int d = d0 + 8 * k;
+      x[s * kU + k] = __ldcg(src + (size_t)s * kSplitU + (size_t)((d >> 5) * 4 + ((d >> 3) & 3)) * 32);
+    }
+#pragma unroll
+  for (int k = 0; k < kU; ++k) {
+    float a[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) a[j] = 0.f;
+#pragma unroll
+    for (int s = 0; s < N; ++s) {
+      const uint32_t w4[4] = {x[s * kU + k].x, x[s * kU + k].y, x[s * kU + k].z, x[s * kU + k].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[j]));
+        a[2 * j] += w[s] * f.x;
+        a[2 * j + 1] += w[s] * f.y;
+      }
+    }
+    *reinterpret_cast<uint4*>(orow + 8 * k) =
+        make_uint4(pack_bf16x2(a[0] * inv, a[1] * inv), pack_bf16x2(a[2] * inv, a[3] * inv),
+                   pack_bf16x2(a[4] * inv, a[5] * inv), pack_bf16x2(a[6] * inv, a[7] * inv));
+  }
 }
 
 template <bool kFp8>
@@ -988,6 +1033,8 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       if (!aborted && half == 0) {
         float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
         *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4) = make_float4(m_run, l_tot, l_nrm, 0.f);
+        // for the merge writers: 1 / (rounded-P sum) of head h
+        reinterpret_cast<float*>(smem + kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
       }
     } else if (!aborted) {
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
@@ -1072,8 +1119,8 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     const int n = p.nsplit;
     const int q = warp & 3;                                  // tensor-memory lane quarter
     const int upper = warp >> 2;                             // 0: softmax warp, 1: helper warp
-    constexpr size_t kSplit4 = (size_t)kH * kDv / 4;         // float4 per split
-    float4* wso = reinterpret_cast<float4*>(p.part_o) + (size_t)b * n * kSplit4;   // [src][q][c][u][lane]
+    constexpr size_t kSplitU = (size_t)kH * kDv / 8;         // 16-byte units (8 fp16) per split
+    uint4* wso = reinterpret_cast<uint4*>(p.part_o) + (size_t)b * n * kSplitU;     // [src][q][c][u][lane]
     const float* wss = p.part_lse + (size_t)b * n * 64 * 4;  // [src][64][4]: m, l, l_pv
     bool failed = merge_failed;
     if (upper) {
@@ -1083,7 +1130,11 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     }
     const bool bad = group_any(failed, 1, 256);
     if (!bad) {
-      float4* mine = wso + (size_t)split * kSplit4 + (size_t)q * (8 * 8 * 32) + lane;
+      // this split's result for the thread's head, normalised by its own
+      // rounded-P sum (a convex combination of value rows) and rounded to
+      // fp16: 11 significant bits, error <= 2^-12 of the largest value
+      const float sc = reinterpret_cast<const float*>(smem + kAuxRow)[16 * q + (lane & 15)];
+      uint4* mine = wso + (size_t)split * kSplitU + (size_t)q * (8 * 4 * 32) + lane;
       const uint32_t olanes = (uint32_t)(32 * q + kLaneO) << 16;
       float o[2][32];
       const int c0 = 4 * upper;
@@ -1099,9 +1150,11 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         const int c = c0 + cc;
         if (ntiles > 0 && cc + 1 < 4) tmem_ld_16x32bx2_x32_h256(tmem + olanes + 32u * (uint32_t)(c + 1), o[(cc + 1) & 1]);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          mine[(c * 8 + u) * 32] = make_float4(o[cc & 1][4 * u], o[cc & 1][4 * u + 1], o[cc & 1][4 * u + 2],
-                                               o[cc & 1][4 * u + 3]);
+        for (int u = 0; u < 4; ++u) {
+          const float* x = &o[cc & 1][8 * u];
+          mine[(c * 4 + u) * 32] = make_uint4(pack_f16x2(x[0] * sc, x[1] * sc), pack_f16x2(x[2] * sc, x[3] * sc),
+                                              pack_f16x2(x[4] * sc, x[5] * sc), pack_f16x2(x[6] * sc, x[7] * sc));
+        }
         if (ntiles > 0 && cc + 1 < 4) tmem_wait_ld();
       }
     }
@@ -1116,10 +1169,14 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     if (!group_any(bad || !ok, 1, 256)) {
       const int hh = 16 * q + (lane & 15);
       const int part = (lane >> 4) + 2 * upper;
-      float mv[16];
+      float mv[16], lr[16], lp[16];
 #pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2)
-        if (s2 < n) mv[s2] = __ldcg(wss + ((size_t)s2 * 64 + hh) * 4);
+      for (int s2 = 0; s2 < 16; ++s2) {
+        if (s2 < n) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
+          mv[s2] = v.x; lr[s2] = v.y; lp[s2] = v.z;
+        }
+      }
       float M = -INFINITY;
 #pragma unroll
       for (int s2 = 0; s2 < 16; ++s2)
@@ -1128,43 +1185,27 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 #pragma unroll
       for (int s2 = 0; s2 < 16; ++s2) {
         if (s2 < n) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
-          const float wgt = mv[s2] > -INFINITY ? ex2(mv[s2] - M) : 0.f;
-          mv[s2] = wgt;                    // from here on: the weight of split s2
-          Lr += wgt * v.y;
-          Lp += wgt * v.z;
+          const float e = mv[s2] > -INFINITY ? ex2(mv[s2] - M) : 0.f;
+          Lr += e * lr[s2];
+          Lp += e * lp[s2];
+          mv[s2] = e * lp[s2];             // from here on: the weight of split s2's normalised result
         }
       }
       const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
       if (split == 0 && part == 0)
         p.lse[(size_t)b * kH + hh] = Lr > 0.f ? (M + log2f(Lr)) * 0.6931471805599453f : -INFINITY;
       if (threadIdx.x == 0) SMLA_TRACE_EV(56);
-      // this thread: columns [col0, col0 + cn / 4), stored by lane
-      // hh % 16 (+16 for dims >= 256) of quarter q of every split
+      // this thread: columns [col0, col0 + cn / 4), 8 per 16-byte unit,
+      // stored by lane hh % 16 (+16 for dims >= 256) of quarter q
       const int cn = kDv / n;
-      const int nv = cn / 16;                                  // float4 per thread (>= 2)
       const int col0 = split * cn + part * (cn / 4);
-      const int hf = col0 >> 8;
-      const float4* src = wso + (size_t)q * (8 * 8 * 32) + (lane & 15) + 16 * hf;
+      const uint4* src = wso + (size_t)q * (8 * 4 * 32) + (lane & 15) + 16 * (col0 >> 8);
       __nv_bfloat16* orow = p.out + ((size_t)b * kH + hh) * kDv + col0;
-#pragma unroll 1
-      for (int v0 = 0; v0 < nv; v0 += 2) {
-        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) {
-          if (s2 < n) {
-            const float wgt = mv[s2];
-            const float4* ss = src + (size_t)s2 * kSplit4;
-            const int d = (col0 & 255) + 4 * v0;              // dim within the half, multiple of 8
-            const float4 x = __ldcg(ss + ((d >> 5) * 8 + ((d >> 2) & 7)) * 32);
-            const float4 y = __ldcg(ss + (((d + 4) >> 5) * 8 + (((d + 4) >> 2) & 7)) * 32);
-            a0.x += wgt * x.x; a0.y += wgt * x.y; a0.z += wgt * x.z; a0.w += wgt * x.w;
-            a1.x += wgt * y.x; a1.y += wgt * y.y; a1.z += wgt * y.z; a1.w += wgt * y.w;
-          }
-        }
-        *reinterpret_cast<uint4*>(orow + 4 * v0) =
-            make_uint4(pack_bf16x2(a0.x * inv, a0.y * inv), pack_bf16x2(a0.z * inv, a0.w * inv),
-                       pack_bf16x2(a1.x * inv, a1.y * inv), pack_bf16x2(a1.z * inv, a1.w * inv));
+      switch (n) {   // 16 loads per thread for every n: all issued before any is used
+        case 2: merge_columns<2>(src, col0 & 255, mv, inv, orow); break;
+        case 4: merge_columns<4>(src, col0 & 255, mv, inv, orow); break;
+        case 8: merge_columns<8>(src, col0 & 255, mv, inv, orow); break;
+        default: merge_columns<16>(src, col0 & 255, mv, inv, orow); break;
       }
       if (threadIdx.x == 0) SMLA_TRACE_EV(62);
     }
@@ -1294,11 +1335,11 @@ static size_t partial_bytes(int batch, int nsplit) {
   return ((o + l + 255) / 256) * 256;
 }
 
-// Workspace of an in-cluster merge: every CTA's O as nsplit column blocks
-// (B * nsplit * 64 * 512 fp32) and its per-head (m, l, l_pv, -) (B * nsplit
+// Workspace of an in-cluster merge: every split's normalised result
+// (B * nsplit * 64 * 512 fp16) and its per-head (m, l, l_pv, -) (B * nsplit
 // * 64 * 4 fp32).
 static size_t cluster_bytes(int batch, int nsplit) {
-  const size_t o = (size_t)batch * nsplit * kH * kDv * 4;
+  const size_t o = (size_t)batch * nsplit * kH * kDv * 2;
   const size_t st = (size_t)batch * nsplit * kH * 4 * 4;
   return ((o + st + 255) / 256) * 256;
 }
@@ -1425,7 +1466,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.cluster = cluster ? 1 : 0;
   prm.part_o = static_cast<float*>(workspace);
   prm.part_lse = n > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                  (size_t)shape->batch * n * kH * kDv * 4)
+                                                  (size_t)shape->batch * n * kH * kDv * (cluster ? 2 : 4))
                        : nullptr;
   prm.batch = shape->batch;
   prm.topk = shape->topk;
