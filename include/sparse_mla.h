@@ -107,10 +107,12 @@ const char* sparse_mla_status_string(smla_status status);
  * With more than one split, sparse_mla_decode merges the splits in one of
  * two ways (sparse_mla_plan_merge tells which).  When nsplit is a power of
  * two no larger than 16 that the device can launch as a thread-block
- * cluster, the CTAs of a sequence form a cluster: each writes its partial
- * result to the workspace, the cluster synchronises, and each CTA reduces
- * one block of output columns -- one kernel.  Otherwise each split writes
- * a partial result and a second (combine) kernel merges them.  An automatic
+ * cluster, the CTAs of a sequence form a cluster: each writes its result,
+ * normalised by its own softmax sum and rounded to fp16 (11 significant
+ * bits; value magnitudes must stay within the fp16 range), to the
+ * workspace, the cluster synchronises, and each CTA reduces one block of
+ * output columns -- one kernel.  Otherwise each split writes an fp32
+ * partial result and a second (combine) kernel merges them.  An automatic
  * plan (shape->nsplit == 0) takes the largest such power of two for which
  * all clusters are resident at once. */
 int32_t sparse_mla_plan_nsplit(const smla_shape* shape);
