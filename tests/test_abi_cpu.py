@@ -87,6 +87,15 @@ def test_bad_shapes_rejected_without_cuda(kw, code):
     assert _decode(shape(**kw)) == code
     assert api.lib.sparse_mla_workspace_size(ctypes.byref(shape(**kw))) == 0
     assert api.lib.sparse_mla_plan_nsplit(ctypes.byref(shape(**kw))) == 0
+    assert api.lib.sparse_mla_plan_merge(ctypes.byref(shape(**kw))) == -1
+    assert api.lib.sparse_mla_decode_static_scratch(ctypes.byref(shape(**kw)), 16, 16, None, None, 16, 0.04,
+                                                    16, 16, None) == code
+
+
+def test_partials_size_formula():
+    # B * nsplit * 64 * (512 + 1) fp32, rounded up to 256 bytes
+    assert api.partials_size(1, 1) == 131328
+    assert api.partials_size(3, 5) == (3 * 5 * 64 * 513 * 4 + 255) // 256 * 256
 
 
 def test_null_and_misaligned_pointers_rejected():
