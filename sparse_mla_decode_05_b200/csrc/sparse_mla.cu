@@ -511,6 +511,13 @@ __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity) {
   return true;
 }
 __device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// Programmatic dependent launch: the grid may start while the previous
+// kernel of the stream is still running (its prologue overlaps that
+// kernel's tail); griddepcontrol.wait blocks until every prerequisite grid
+// has completed and its memory is visible, launch_dependents lets the next
+// grid start early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 // every thread of every CTA of the cluster (executed unconditionally by all)
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -523,9 +530,6 @@ __device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, u
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(sdst),
                "l"(gsrc), "r"(bytes), "r"(bar)
                : "memory");
-}
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // In-cluster merge, final step for one thread: columns [d0, d0 + 64 / N * 4)
@@ -634,6 +638,9 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   // Cluster launch: the barriers of every CTA are initialised before any
   // CTA of the cluster can arrive on them remotely.
   if (p.cluster) cluster_sync_all();
+  // nothing above reads or writes global memory: with programmatic
+  // dependent launch all of it overlapped the previous kernel
+  grid_dep_wait();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kAuxTmem);
   SMLA_TRACE_EV(1);
@@ -642,9 +649,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   if (warp >= kWarpIdx && warp < kWarpIdx + kIdxWarps) {
     // ------------------------------------------------------------ index warps
     // Resolve each tile's 64 entries to physical rows (and fp8 row scales)
-    // into the kRing-deep ring ahead of the loaders, and pull the rows into
-    // L2.  Warp k handles tiles t = k, k+4, ... (ring slot k), so four tiles'
-    // lookups are in flight at once.
+    // into the kRing-deep ring ahead of the loaders.  Warp k handles tiles
+    // t = k, k+4, ... (ring slot k), so four tiles' lookups are in flight at
+    // once.  (Pulling the rows into L2 ahead of the loaders, one bulk
+    // prefetch per row, measured slower: it queues on the copy engine.)
     auto idx_at = [&](int t, int j) -> int {
       const int pos = tok_begin + t * kTile + j;
       return (t < ntiles && pos < tok_end) ? __ldg(p.indices + (size_t)b * p.topk + pos) : -1;
@@ -665,9 +673,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     }
     // Software pipeline over this warp's tiles (step S = 4), every load
     // consumed one iteration after it was issued: index of tile t+3S, page
-    // entry of t+2S, row scale of t+S (and the rows of t+S pulled into L2),
-    // then tile t is published.
-    constexpr uint32_t kRowBytes = kFp8 ? kRowBytesFp8 : kRowBytesBf16;
+    // entry of t+2S, row scale of t+S, then tile t is published.
     constexpr int S = kIdxWarps;
     int i2_0 = idx_at(kw + 2 * S, lane), i2_1 = idx_at(kw + 2 * S, lane + 32);                 // tile t+2S
     int r1_0 = row_of(idx_at(kw + S, lane)), r1_1 = row_of(idx_at(kw + S, lane + 32));         // tile t+S
@@ -677,8 +683,6 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       c0_0 = r0_0 >= 0 ? __ldg(p.kv_row_scale + r0_0) : 0.f;
       c0_1 = r0_1 >= 0 ? __ldg(p.kv_row_scale + r0_1) : 0.f;
     }
-    if (r0_0 >= 0) prefetch_l2(p.kv + (size_t)r0_0 * kRowBytes, kRowBytes);
-    if (r0_1 >= 0) prefetch_l2(p.kv + (size_t)r0_1 * kRowBytes, kRowBytes);
     for (int t = kw; t < ntiles; t += S) {
       const int rs = t % kRing;
       float c1_0 = 0.f, c1_1 = 0.f;
@@ -686,8 +690,6 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         c1_0 = r1_0 >= 0 ? __ldg(p.kv_row_scale + r1_0) : 0.f;
         c1_1 = r1_1 >= 0 ? __ldg(p.kv_row_scale + r1_1) : 0.f;
       }
-      if (r1_0 >= 0) prefetch_l2(p.kv + (size_t)r1_0 * kRowBytes, kRowBytes);
-      if (r1_1 >= 0) prefetch_l2(p.kv + (size_t)r1_1 * kRowBytes, kRowBytes);
       const int r2_0 = row_of(i2_0), r2_1 = row_of(i2_1);
       const int i3_0 = idx_at(t + 3 * S, lane), i3_1 = idx_at(t + 3 * S, lane + 32);
       const bool fail = t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1);
@@ -761,7 +763,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         for (int u = 0; u < 16; ++u) rows[u] = s_row[rs * 64 + 4 * u + (lane >> 3)];
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) rows[u] = s_row[rs * 64 + 8 * (4 * lw + u) + (lane >> 2)];
+        for (int u = 0; u < 8; ++u) rows[u] = s_row[rs * 64 + 4 * (8 * lw + u) + (lane >> 3)];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
@@ -788,17 +790,22 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
       } else {
         if (lt == 0 && t < 8) SMLA_TRACE_EV(48 + t);
-        // each warp instruction covers eight 64-byte row segments; codes go
-        // to the first chunk of their bf16 destination (see the convert warps)
-        const int sub = lane & 3;
+        // each warp instruction covers four whole 128-byte row segments
+        // (a row is 4.5 segments); 16-code chunk c of a row goes to the first
+        // chunk of its bf16 destination (atom c / 4, see the convert warps)
+        const int j = lane & 7;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int tok = 8 * (4 * lw + u) + (lane >> 2);
+        for (int u = 0; u < 8; ++u) {
+          const int tok = 4 * (8 * lw + u) + (lane >> 3);
           const int row = rows[u];
-          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8 + sub * 16;
+          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8;
 #pragma unroll
-          for (int a = 0; a < kAtoms; ++a)
-            cp_async_16(tbase + a * kAtomBytes + sw128_off(tok, 2 * sub), src + a * 64, row >= 0 ? 16u : 0u);
+          for (int sg = 0; sg < 5; ++sg) {
+            const int c = 8 * sg + j;
+            if (c < kRowBytesFp8 / 16)
+              cp_async_16(tbase + (c >> 2) * kAtomBytes + sw128_off(tok, 2 * (c & 3)), src + c * 16,
+                          row >= 0 ? 16u : 0u);
+          }
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_RAW + stage));
       }
@@ -1016,6 +1023,9 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       if (threadIdx.x == 0 && i < 8) SMLA_TRACE_EV(32 + i);
     }
     // ---------------------------------------------------------- epilogue
+    // this CTA's tiles are done: the next kernel of the stream may start
+    // on idle SMs (it waits for this grid's completion before reading)
+    if (threadIdx.x == 0) grid_dep_launch();
     if (!aborted && ntiles > 0) {
       // PV(n-2) then PV(n-1): each wait is at most one phase ahead
       if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + (ntiles & 1)), ((ntiles - 2) >> 1) & 1)) aborted = true;
@@ -1227,6 +1237,8 @@ __global__ void __launch_bounds__(128) smla_combine_kernel(const float* __restri
                                                            const float* __restrict__ part_lse,
                                                            __nv_bfloat16* __restrict__ out,
                                                            float* __restrict__ lse, int nsplit) {
+  grid_dep_wait();       // the split kernel's partials are complete
+  grid_dep_launch();
   const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
   const float* pl = part_lse + (size_t)b * nsplit * kH + h;
   float mx = -INFINITY;
@@ -1411,23 +1423,27 @@ static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
   auto kern = smla_split_kernel<kFp8>;
   cudaError_t e = ensure_smem_attr<kFp8>();
   if (e != cudaSuccess) return e;
-  dim3 grid(prm.nsplit, prm.batch);
-  if (!prm.cluster) {
-    kern<<<grid, Cfg<kFp8>::kThreads, kSmemBytes, stream>>>(prm);
-    return cudaGetLastError();
+  // programmatic dependent launch (the kernel waits for its prerequisites
+  // itself), and for an in-cluster merge the cluster of nsplit CTAs
+  cudaLaunchAttribute at[2];
+  int na = 0;
+  at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (prm.cluster) {
+    at[na].id = cudaLaunchAttributeClusterDimension;
+    at[na].val.clusterDim.x = prm.nsplit;
+    at[na].val.clusterDim.y = 1;
+    at[na].val.clusterDim.z = 1;
+    ++na;
   }
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = prm.nsplit;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
+  cfg.gridDim = dim3(prm.nsplit, prm.batch);
   cfg.blockDim = dim3(Cfg<kFp8>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
@@ -1486,8 +1502,18 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
 static smla_status run_combine(int batch, int nsplit, const float* part_o, const float* part_lse, void* out,
                                float* lse, cudaStream_t stream) {
   dim3 grid(kH, batch);
-  smla_combine_kernel<<<grid, 128, 0, stream>>>(part_o, part_lse, static_cast<__nv_bfloat16*>(out), lse, nsplit);
-  return cudaGetLastError() == cudaSuccess ? SMLA_OK : SMLA_ERR_CUDA;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.stream = stream;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, smla_combine_kernel, part_o, part_lse,
+                                           static_cast<__nv_bfloat16*>(out), lse, nsplit);
+  return e == cudaSuccess ? SMLA_OK : SMLA_ERR_CUDA;
 }
 
 // Device address of g_static_scratch on the current device, looked up once

@@ -341,6 +341,44 @@ def test_cuda_graph_replay_bit_identical(name):
     del g
 
 
+def test_cuda_graph_back_to_back_calls():
+    """Several decode calls in one CUDA graph (each launch may start before
+    the previous one ends: programmatic dependent launch), on different
+    inputs and plans: partials + combine, in-cluster merge, one split, fp8.
+    Replays equal the eager results bit for bit."""
+    a = api()
+    ws = [inputs.flat_per_seq(2, 2048, 700, seed=91),          # explicit 3 splits: combine kernel
+          inputs.flat_per_seq(2, 2048, 700, seed=92),          # 4 splits: in-cluster merge
+          inputs.paged_fp8(3, 1024, 64, 300, seed=93),         # fp8, planned
+          inputs.flat_per_seq(4, 1000, 64, seed=94)]           # one tile: one split
+    nsplits = [3, 4, 0, 0]
+    plans, eager = [], []
+    for w, n in zip(ws, nsplits):
+        d = Dev(w)
+        pl = a.DecodePlan(d.q, d.kv, d.indices, w.scale, kv_row_scale=d.kv_row_scale, page_table=d.page_table,
+                          page_size=w.page_size, nsplit=n)
+        pl.run()
+        torch.cuda.synchronize()
+        eager.append((pl.out.clone(), pl.lse.clone()))
+        plans.append((d, pl))
+    assert plans[0][1].nsplit == 3 and not plans[0][1].clustered     # combine kernel path
+    assert plans[1][1].nsplit == 4 and plans[1][1].clustered         # in-cluster merge
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _, pl in plans:
+            pl.run(torch.cuda.current_stream().cuda_stream)
+    for _, pl in plans:
+        pl.out.zero_()
+        pl.lse.zero_()
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    for (_, pl), (o, l) in zip(plans, eager):
+        assert torch.equal(pl.out.view(torch.int16), o.view(torch.int16))
+        assert torch.equal(pl.lse.view(torch.int32), l.view(torch.int32))
+    del g
+
+
 def test_workspace_checks():
     w = inputs.flat_per_seq(2, 1000, 300, seed=1)
     d = Dev(w)
