@@ -47,6 +47,8 @@ import numpy as np
 __all__ = [
     "bf16_bits_to_f64",
     "e4m3fn_to_f64",
+    "ue8m0_to_f64",
+    "dsv4_rows_f64",
     "f64_to_bf16_bits_rne",
     "resolve_rows",
     "gather_rows_f64",
@@ -118,6 +120,48 @@ def f64_to_bf16_bits_rne(x: np.ndarray) -> np.ndarray:
     return out
 
 
+def ue8m0_to_f64(e: np.ndarray) -> np.ndarray:
+    """UE8M0 scale bytes (OCP microscaling E8M0: an unsigned biased exponent,
+    no sign, no mantissa) -> 2^(e - 127); the byte 0xFF is NaN."""
+    e = np.asarray(e).astype(np.int64)
+    out = np.ldexp(1.0, e - 127)
+    return np.where(e == 255, np.nan, out)
+
+
+# DeepSeek-V4 paged cache layout ([Design] "The Agent Reasoning" -> "Cache
+# Layout Understanding"; reading: a 64-token page holds the 64 token slots of
+# 576 bytes first, then the 64 scale blocks of 8 bytes, 584 bytes per token):
+#   slot i, bytes [576 i, 576 i + 448): 448 fp8 e4m3fn codes, the "nope" dims
+#   slot i, bytes [576 i + 448, 576 (i+1)): 64 bf16 values, the "rope" dims
+#   bytes [36864 + 8 i, 36864 + 8 i + 7): UE8M0 scale of nope group g (dims
+#   64 g .. 64 g + 63), g = 0..6; byte 7 unused
+DSV4_PAGE_TOKENS = 64
+DSV4_SLOT_BYTES = 576
+DSV4_PAGE_BYTES = 64 * 584          # 37,376
+DSV4_NOPE = 448
+DSV4_ROPE = 64
+
+
+def dsv4_rows_f64(pages: np.ndarray, rows: np.ndarray) -> np.ndarray:
+    """Decode physical rows (page * 64 + slot) of a DeepSeek-V4 paged cache
+    (uint8 [num_pages, 37376]) to float64 [n, 512]: the 448 nope dims, each
+    e4m3fn code times its group's UE8M0 scale, then the 64 bf16 rope dims.
+    The whole 512-dim row is both key and value ([Design] "Kernel Structure
+    Analysis": the output accumulates nope and rope values)."""
+    pages = np.asarray(pages, dtype=np.uint8)
+    rows = np.asarray(rows, dtype=np.int64)
+    page, slot = rows // DSV4_PAGE_TOKENS, rows % DSV4_PAGE_TOKENS
+    base = slot * DSV4_SLOT_BYTES
+    codes = pages[page[:, None], base[:, None] + np.arange(DSV4_NOPE)]
+    rope_lo = pages[page[:, None], (base + DSV4_NOPE)[:, None] + 2 * np.arange(DSV4_ROPE)].astype(np.uint16)
+    rope_hi = pages[page[:, None], (base + DSV4_NOPE + 1)[:, None] + 2 * np.arange(DSV4_ROPE)].astype(np.uint16)
+    rope = bf16_bits_to_f64(rope_lo | (rope_hi << 8))
+    sb = DSV4_PAGE_TOKENS * DSV4_SLOT_BYTES + 8 * slot
+    scales = ue8m0_to_f64(pages[page[:, None], sb[:, None] + np.arange(DSV4_NOPE // 64)])
+    nope = e4m3fn_to_f64(codes) * np.repeat(scales, 64, axis=1)
+    return np.concatenate([nope, rope], axis=1)
+
+
 # --------------------------------------------------------------------------
 # Index resolution.
 # --------------------------------------------------------------------------
@@ -158,7 +202,10 @@ def gather_rows_f64(kv: np.ndarray, rows: np.ndarray, *, kv_format: str,
     kv_format "bf16": kv holds bf16 bit patterns (uint16).
     kv_format "fp8_e4m3_rowscale": kv holds e4m3fn codes (uint8); each row is
     multiplied by its fp32 row scale (in fp64).
+    kv_format "dsv4_paged": kv holds DeepSeek-V4 pages (uint8 [pages, 37376]).
     """
+    if kv_format == "dsv4_paged":
+        return dsv4_rows_f64(kv, rows)
     raw = kv[rows]
     if kv_format == "bf16":
         return bf16_bits_to_f64(raw)
@@ -206,14 +253,20 @@ def sparse_mla_decode(q_bits: np.ndarray, kv: np.ndarray, indices: np.ndarray,
     """
     q_bits = np.asarray(q_bits)
     B, H, d_qk = q_bits.shape
-    if kv.shape[1] != d_qk:
-        raise ValueError("row width differs from the query width")
+    if kv_format == "dsv4_paged":
+        if d_qk != DSV4_NOPE + DSV4_ROPE or kv.shape[1] != DSV4_PAGE_BYTES:
+            raise ValueError("DeepSeek-V4 pages need a 512-dim query and 37376-byte pages")
+        num_rows = kv.shape[0] * DSV4_PAGE_TOKENS
+    else:
+        if kv.shape[1] != d_qk:
+            raise ValueError("row width differs from the query width")
+        num_rows = kv.shape[0]
     out = np.full((B, H, d_v), np.nan)
     lse = np.full((B, H), np.nan)
     for b in (range(B) if seqs is None else seqs):
         rows = resolve_rows(indices[b],
                             page_table_row=None if page_table is None else page_table[b],
-                            page_size=page_size, num_rows=kv.shape[0])
+                            page_size=page_size, num_rows=num_rows)
         rows = rows[rows >= 0]
         k = gather_rows_f64(kv, rows, kv_format=kv_format, row_scale=kv_row_scale)
         qh = bf16_bits_to_f64(q_bits[b])

@@ -54,6 +54,7 @@ class Workload:
     page_size: int = 0
     d_v: int = D_V
     meta: dict = dataclasses.field(default_factory=dict)
+    layout: str = ""                           # "dsv4": DeepSeek-V4 pages (uint8 [pages, 37376])
 
     @property
     def batch(self) -> int:
@@ -65,6 +66,8 @@ class Workload:
 
     @property
     def kv_format(self) -> str:
+        if self.layout == "dsv4":
+            return "dsv4_paged"
         return "fp8_e4m3_rowscale" if self.kv.dtype == torch.uint8 else "bf16"
 
     def valid_count(self) -> int:
@@ -182,6 +185,46 @@ def paged_fp8(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: i
                     page_size=page_size,
                     meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages,
                               topk=topk, seed=seed))
+
+
+DSV4_PAGE_BYTES = 64 * 584          # 64 slots of 576 bytes, then 64 scale blocks of 8 bytes
+
+
+def paged_dsv4(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: int,
+               name: str = "paged_dsv4") -> Workload:
+    """DeepSeek-V4 paged cache: 64-token pages of 37,376 bytes.  Slot i holds
+    448 fp8 e4m3fn "nope" codes then 64 bf16 "rope" values (576 bytes);
+    after the 64 slots come 64 scale blocks of 8 bytes, 7 UE8M0 exponents
+    (one per 64 nope dims) and a zero byte.  Values are N(0,1); a group's
+    scale is the power of two 2^ceil(log2(amax / 448)), so every code is in
+    range.  q is [B, 64, 512] (448 nope + 64 rope dims); indices are logical
+    positions through a page table (a slice of one random permutation of
+    all pages per sequence)."""
+    pps = rows_per_seq // 64
+    if B * pps > total_pages:
+        raise ValueError("not enough pages for distinct page tables")
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(gen, (B, H, 512))
+    pages = torch.zeros((total_pages, DSV4_PAGE_BYTES), dtype=torch.uint8)
+    for p0 in range(0, total_pages, 256):
+        p1 = min(total_pages, p0 + 256)
+        n = (p1 - p0) * 64
+        nope = torch.randn((n, 448), generator=gen, dtype=torch.float32).view(n, 7, 64)
+        amax = nope.abs().amax(dim=2).clamp_min(1e-30)
+        e = torch.ceil(torch.log2(amax / 448.0))
+        codes = (nope / torch.exp2(e)[:, :, None]).view(n, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        rope = torch.randn((n, 64), generator=gen, dtype=torch.float32).to(torch.bfloat16).view(torch.uint8)
+        slots = torch.cat([codes, rope.view(n, 128)], dim=1).view(p1 - p0, 64 * 576)
+        sc = torch.zeros((n, 8), dtype=torch.uint8)
+        sc[:, :7] = (e + 127).to(torch.uint8)
+        pages[p0:p1, :64 * 576] = slots
+        pages[p0:p1, 64 * 576:] = sc.view(p1 - p0, 64 * 8)
+    perm = rng.permutation(total_pages)[: B * pps].reshape(B, pps)
+    idx = np.stack([_distinct(rng, rows_per_seq, topk) for _ in range(B)])
+    return Workload(name=name, q=q, kv=pages, indices=torch.from_numpy(idx.astype(np.int32)),
+                    page_table=torch.from_numpy(perm.astype(np.int32)), page_size=64, layout="dsv4",
+                    meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages, topk=topk, seed=seed))
 
 
 CONFIG_NAMES = ("c1", "c2", "c3", "c4a", "c4b", "c5")

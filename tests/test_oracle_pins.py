@@ -366,3 +366,84 @@ def test_pins_accept_the_oracle():
                                   "no_scale", "sign", "value_tail", "lse_no_max"])
 def test_pins_reject_planted_mistakes(kind):
     assert not _pins_pass(_mutant(kind))
+
+
+# ------------------------------------------------ DeepSeek-V4 paged layout
+def test_ue8m0_decode_all_codes():
+    e = np.arange(256)
+    got = ref.ue8m0_to_f64(e)
+    for v in range(255):
+        assert got[v] == math.ldexp(1.0, v - 127)
+    assert np.isnan(got[255])
+
+
+def _hand_page(mistake=None):
+    """Page 2 of 3, slot 5, written byte by byte; returns (pages, row, want)."""
+    pages = np.zeros((3, 64 * 584), np.uint8)
+    slot, page = 5, 2
+    base = 576 * slot
+    codes = np.full(448, 0x38, np.uint8)            # e4m3fn 0x38 = 1.0
+    codes[0] = 0xC0                                 # -2.0
+    codes[64] = 0x30                                # 0.5
+    codes[447] = 0x01                               # 2^-9 (smallest subnormal)
+    pages[page, base:base + 448] = codes
+    rope = np.zeros(64, np.uint16)
+    rope[0], rope[63] = 0x3FC0, 0xBE80              # bf16 1.5, -0.25
+    pages[page, base + 448:base + 576] = rope.view(np.uint8)     # little-endian bytes
+    sc = np.full(7, 127, np.uint8)
+    sc[0], sc[1], sc[6] = 128, 126, 130             # x2, x0.5, x8
+    pages[page, 64 * 576 + 8 * slot:64 * 576 + 8 * slot + 7] = sc
+    want = np.ones(512)
+    want[0:64] = 2.0
+    want[0] = -4.0
+    want[64:128] = 0.5
+    want[64] = 0.25
+    want[384:448] = 8.0
+    want[447] = 8.0 * 2.0 ** -9
+    want[448:512] = 0.0
+    want[448], want[511] = 1.5, -0.25
+    rows_fn = ref.dsv4_rows_f64
+    if mistake == "scale_group_shift":
+        def rows_fn(p, r):
+            v = ref.dsv4_rows_f64(p, r)
+            nope = ref.e4m3fn_to_f64(p[r // 64][:, (r % 64)[0] * 576:(r % 64)[0] * 576 + 448])
+            sc_ = ref.ue8m0_to_f64(p[r // 64][:, 64 * 576 + 8 * (r % 64)[0]:64 * 576 + 8 * (r % 64)[0] + 7])
+            v[:, :448] = nope * np.repeat(np.roll(sc_, 1, axis=1), 64, axis=1)
+            return v
+    if mistake == "rope_big_endian":
+        def rows_fn(p, r):
+            v = ref.dsv4_rows_f64(p, r)
+            b = p[r // 64][:, (r % 64)[0] * 576 + 448:(r % 64)[0] * 576 + 576].astype(np.uint16)
+            v[:, 448:] = ref.bf16_bits_to_f64((b[:, 0::2] << 8) | b[:, 1::2])
+            return v
+    if mistake == "scale_on_rope":
+        def rows_fn(p, r):
+            v = ref.dsv4_rows_f64(p, r)
+            v[:, 448:] *= 2.0
+            return v
+    return pages, np.array([page * 64 + slot]), want, rows_fn
+
+
+@pytest.mark.parametrize("mistake", [None, "scale_group_shift", "rope_big_endian", "scale_on_rope"])
+def test_dsv4_hand_built_page(mistake):
+    pages, row, want, rows_fn = _hand_page(mistake)
+    got = rows_fn(pages, row)[0]
+    assert np.array_equal(got, want) == (mistake is None)
+
+
+def test_dsv4_decode_equals_the_plain_path_on_decoded_rows():
+    """The paged DeepSeek-V4 decode equals the (torch-pinned) bf16 path run on
+    a flat pool holding the decoded rows: e4m3fn value x power of two and
+    bf16 rope are exact in bf16, and V is the whole 512-dim row."""
+    w = inputs.paged_dsv4(3, 512, 32, 200, seed=12)
+    pages = w.kv.numpy()
+    idx = w.indices.numpy()
+    pt = w.page_table.numpy()
+    o, l = ref.sparse_mla_decode(w.np_q_bits(), pages, idx, w.scale, kv_format="dsv4_paged",
+                                 page_table=pt, page_size=64)
+    n_rows = pages.shape[0] * 64
+    flat = ref.dsv4_rows_f64(pages, np.arange(n_rows))
+    flat_bits = ref.f64_to_bf16_bits_rne(flat)
+    assert np.array_equal(ref.bf16_bits_to_f64(flat_bits), flat)          # exact in bf16
+    of, lf = ref.sparse_mla_decode(w.np_q_bits(), flat_bits, idx, w.scale, d_v=512, page_table=pt, page_size=64)
+    assert np.allclose(o, of, atol=1e-12, rtol=0) and np.allclose(l, lf, atol=1e-12, rtol=0)
