@@ -391,7 +391,7 @@ def main():
     per_config = None
     if rank == 0 and world == 1 and not args.no_per_config:
         per_config = []
-        for name in inputs.CONFIG_NAMES:
+        for name in inputs.CONFIG_NAMES + inputs.EXTRA_NAMES:
             wc = w if name == args.workload else inputs.make_config(name)
             rc = r if name == args.workload else Runner(wc, dev)
             tms = time_device(rc.decode, 30, 3, flush, stream)

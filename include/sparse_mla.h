@@ -69,12 +69,26 @@ typedef enum {
 
 typedef enum {
   SMLA_KV_BF16 = 0,             /* cache rows: bf16 [num_kv_rows, 576]      */
-  SMLA_KV_FP8_E4M3_ROWSCALE = 1 /* cache rows: OCP fp8 e4m3fn codes
+  SMLA_KV_FP8_E4M3_ROWSCALE = 1, /* cache rows: OCP fp8 e4m3fn codes
                                    [num_kv_rows, 576] (uint8), and one fp32
                                    scale per row: value = decode(code)*scale */
+  SMLA_KV_DSV4_PAGED = 2        /* DeepSeek-V4 paged cache ([Design] "The
+                                   Agent Reasoning" -> "Cache Layout
+                                   Understanding"): pages of 64 token slots,
+                                   37,376 bytes each.  Slot i: bytes
+                                   [576 i, 576 i + 448) = 448 e4m3fn "nope"
+                                   codes, then 64 bf16 "rope" values; bytes
+                                   [36864 + 8 i, +7) = UE8M0 scales (2^(e-127))
+                                   of the nope dims 64 g .. 64 g + 63, g < 7.
+                                   The 512-dim row (448 nope x scale, 64 rope)
+                                   is both key and value: d_qk = d_v = 512,
+                                   q is [B, 64, 512].  Paged only (page_size
+                                   64); num_kv_rows = 64 * pages; no
+                                   kv_row_scale. */
 } smla_kv_dtype;
 
-/* Problem description.  num_heads must be 64, d_qk 576, d_v 512. */
+/* Problem description.  num_heads must be 64, d_v 512, d_qk 576 (512 for
+ * SMLA_KV_DSV4_PAGED). */
 typedef struct {
   int32_t batch;          /* B >= 1: sequences, one query token each          */
   int32_t num_heads;      /* H = 64                                            */
@@ -131,11 +145,15 @@ size_t sparse_mla_workspace_size(const smla_shape* shape);
 
 /* One decode step: the split kernel, plus the combine kernel when the plan
  * merges its splits through a second kernel (sparse_mla_plan_merge == 2).
- *   q            [B, 64, 576] bf16
- *   kv_cache     [num_kv_rows, 576] bf16, or uint8 e4m3fn codes
+ *   q            [B, 64, 576] bf16 ([B, 64, 512] for SMLA_KV_DSV4_PAGED)
+ *   kv_cache     [num_kv_rows, 576] bf16, or uint8 e4m3fn codes, or
+ *                [num_kv_rows / 64, 37376] uint8 DeepSeek-V4 pages
  *   kv_row_scale [num_kv_rows] fp32 for SMLA_KV_FP8_E4M3_ROWSCALE, else NULL
  *   page_table   [B, pages_per_seq] int32 when page_size > 0, else NULL
- *   indices      [B, topk] int32, -1 = padding (anywhere in the list)
+ *   indices      [B, topk] int32, -1 = padding (anywhere in the list).  An
+ *                entry at or past pages_per_seq * page_size (paged), or
+ *                that resolves to a row outside [0, num_kv_rows), is read
+ *                as padding and sets bit 2 of the device error word.
  *   scale        softmax scale (e.g. 1/sqrt(576))
  *   out          [B, 64, 512] bf16   (written)
  *   lse          [B, 64] fp32        (written; natural log, scale included)
@@ -181,7 +199,8 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
 /* Reads and clears the library's device error word on the current device
  * (a synchronous device-to-host copy: call it outside timed or captured
  * regions).  *code receives the raw word (0 = no error; bit 0: a kernel gave
- * up waiting on a pipeline barrier).  Returns SMLA_ERR_DEVICE_TIMEOUT if
+ * up waiting on a pipeline barrier; bit 1: misaligned shared memory window;
+ * bit 2: an index entry named no row of the pool and was read as padding).  Returns SMLA_ERR_DEVICE_TIMEOUT if
  * the word was non-zero, SMLA_OK if zero, SMLA_ERR_CUDA on a copy failure. */
 smla_status sparse_mla_get_device_error(uint32_t* code);
 

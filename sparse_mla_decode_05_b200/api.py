@@ -16,7 +16,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsparse_mla.so")
 
 H, D_QK, D_V, TILE = 64, 576, 512, 64
-KV_BF16, KV_FP8_E4M3_ROWSCALE = 0, 1
+KV_BF16, KV_FP8_E4M3_ROWSCALE, KV_DSV4_PAGED = 0, 1, 2
+DSV4_PAGE_BYTES, DSV4_D_QK = 37376, 512   # DeepSeek-V4 page: 64 x 576 slot bytes + 64 x 8 scale bytes
 
 STATUS = {0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARG", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_WORKSPACE",
           4: "SMLA_ERR_CUDA", 5: "SMLA_ERR_DEVICE_TIMEOUT"}
@@ -78,15 +79,22 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def make_shape(batch: int, topk: int, num_kv_rows: int, *, fp8: bool = False, page_size: int = 0,
-               pages_per_seq: int = 0, nsplit: int = 0) -> SmlaShape:
-    return SmlaShape(batch, H, D_QK, D_V, topk, KV_FP8_E4M3_ROWSCALE if fp8 else KV_BF16,
+def make_shape(batch: int, topk: int, num_kv_rows: int, *, fp8: bool = False, dsv4: bool = False,
+               page_size: int = 0, pages_per_seq: int = 0, nsplit: int = 0) -> SmlaShape:
+    kind = KV_DSV4_PAGED if dsv4 else (KV_FP8_E4M3_ROWSCALE if fp8 else KV_BF16)
+    return SmlaShape(batch, H, DSV4_D_QK if dsv4 else D_QK, D_V, topk, kind,
                      num_kv_rows, page_size, pages_per_seq, nsplit, 0)
 
 
+def is_dsv4(kv) -> bool:
+    """A DeepSeek-V4 paged cache: uint8 [pages, 37376]."""
+    return kv.dtype == torch.uint8 and kv.dim() == 2 and kv.shape[1] == DSV4_PAGE_BYTES
+
+
 def shape_for(q, kv, indices, *, page_table=None, page_size: int = 0, nsplit: int = 0) -> SmlaShape:
-    return make_shape(q.shape[0], indices.shape[1], kv.shape[0], fp8=(kv.dtype == torch.uint8),
-                      page_size=page_size,
+    dsv4 = is_dsv4(kv)
+    return make_shape(q.shape[0], indices.shape[1], kv.shape[0] * (64 if dsv4 else 1),
+                      fp8=(kv.dtype == torch.uint8 and not dsv4), dsv4=dsv4, page_size=page_size,
                       pages_per_seq=0 if page_table is None else page_table.shape[1], nsplit=nsplit)
 
 
@@ -105,13 +113,21 @@ def workspace_size(shape: SmlaShape) -> int:
 
 
 def _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size):
-    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[1:] != (H, D_QK):
-        raise ValueError("q must be bf16 [B, 64, 576]")
-    if kv.dim() != 2 or kv.shape[1] != D_QK or kv.dtype not in (torch.bfloat16, torch.uint8):
-        raise ValueError("kv must be [N, 576] bf16 or uint8 (fp8 e4m3fn codes)")
+    dsv4 = is_dsv4(kv)
+    d_qk = DSV4_D_QK if dsv4 else D_QK
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[1:] != (H, d_qk):
+        raise ValueError(f"q must be bf16 [B, 64, {d_qk}]")
+    if not dsv4 and (kv.dim() != 2 or kv.shape[1] != D_QK or kv.dtype not in (torch.bfloat16, torch.uint8)):
+        raise ValueError("kv must be [N, 576] bf16 or uint8 (fp8 e4m3fn codes), or uint8 [pages, 37376] "
+                         "DeepSeek-V4 pages")
     if indices.dtype != torch.int32 or indices.dim() != 2 or indices.shape[0] != q.shape[0]:
         raise ValueError("indices must be int32 [B, topk]")
-    if kv.dtype == torch.uint8 and (kv_row_scale is None or kv_row_scale.dtype != torch.float32):
+    if dsv4:
+        if kv_row_scale is not None:
+            raise ValueError("DeepSeek-V4 pages carry their own scales: kv_row_scale must be None")
+        if page_size != 64:
+            raise ValueError("DeepSeek-V4 pages are paged: page_size must be 64")
+    elif kv.dtype == torch.uint8 and (kv_row_scale is None or kv_row_scale.dtype != torch.float32):
         raise ValueError("fp8 cache needs float32 kv_row_scale [N]")
     if page_size and (page_table is None or page_table.dtype != torch.int32):
         raise ValueError("paged cache needs int32 page_table [B, pages_per_seq]")

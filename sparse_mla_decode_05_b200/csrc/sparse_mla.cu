@@ -98,10 +98,16 @@ constexpr int kAuxBars = kSmemAux;
 constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
 constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
 constexpr int kAuxRsc = kAuxRow + kRing * 64 * 4;   // f32  [kRing][64] fp8 row scales
-constexpr int kAuxEnd = kAuxRsc + kRing * 64 * 4;
+constexpr int kAuxDsc = kAuxRsc + kRing * 64 * 4;   // u64  [kRing][64] DeepSeek-V4 scale blocks
+constexpr int kAuxEnd = kAuxDsc + kRing * 64 * 8;
 constexpr int kSmemBytes = kAuxEnd;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
-static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0, "aux arrays are read as 16-byte vectors");
+static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxDsc % 16 == 0, "aux arrays are read as vectors");
+// DeepSeek-V4 page: 64 slots of 576 bytes (448 e4m3fn codes, 64 bf16), then
+// 64 scale blocks of 8 bytes (7 UE8M0 exponents, one per 64 code dims)
+constexpr int kDsv4Slot = 576, kDsv4Nope = 448;
+constexpr int kDsv4ScaleOff = 64 * kDsv4Slot;       // 36,864
+constexpr int kDsv4Page = kDsv4ScaleOff + 64 * 8;   // 37,376
 
 // Tensor memory (512 columns x 128 lanes).  Each warp quarter (32 lanes)
 // holds 16 heads; an M=64 operand or accumulator uses lanes 0-15 or 16-31
@@ -136,10 +142,15 @@ constexpr long long kWaitLimitCycles = 4000000000ll;
 // codes: two warps), then, for fp8 only, eight warps that convert the codes
 // to bf16 in place
 constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kIdxWarps = 4, kWarpLoad0 = kWarpIdx + kIdxWarps;
-template <bool kFp8>
+// cache layouts the split kernel is instantiated for
+constexpr int kKindBf16 = 0;   // bf16 rows [N, 576]
+constexpr int kKindFp8 = 1;    // e4m3fn rows [N, 576] + one fp32 scale per row
+constexpr int kKindDsv4 = 2;   // DeepSeek-V4 pages: 448 e4m3fn + UE8M0 group scales, 64 bf16 rope
+template <int kKind>
 struct Cfg {
-  static constexpr int kCopyWarps = kFp8 ? 2 : 4;
-  static constexpr int kCvtWarps = kFp8 ? 8 : 0;
+  static constexpr bool kConv = kKind != kKindBf16;     // codes converted to bf16 by convert warps
+  static constexpr int kCopyWarps = kConv ? 2 : 4;
+  static constexpr int kCvtWarps = kConv ? 8 : 0;
   static constexpr int kCopyThreads = kCopyWarps * 32;
   static constexpr int kLoadWarps = kCopyWarps + kCvtWarps;
   static constexpr int kThreads = (kWarpLoad0 + kLoadWarps) * 32;
@@ -158,6 +169,7 @@ struct SplitParams {
   int batch, topk, nsplit, ntiles_total;
   int cluster;                 // 1: the nsplit CTAs of a sequence form a cluster and reduce on chip
   int page_size, pages_per_seq;
+  int num_kv_rows;             // rows in the pool (64 x pages when paged)
   float scale_log2;            // scale * log2(e)
 };
 
@@ -301,6 +313,21 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t& lo, uint3
   lo = bf16x2_mul(b0, kTwo120);
   hi = bf16x2_mul(b1, kTwo120);
 }
+// The same, times a power of two given as a bf16x2 pair s2 (both halves
+// equal): the exact code value first, then one more rounding multiply,
+// exact whenever the product is a bf16 normal number.
+__device__ __forceinline__ void e4m3x4_to_bf16x4_scaled(uint32_t w, uint32_t s2, uint32_t& lo, uint32_t& hi) {
+  e4m3x4_to_bf16x4(w, lo, hi);
+  lo = bf16x2_mul(lo, s2);
+  hi = bf16x2_mul(hi, s2);
+}
+// UE8M0 exponent byte e (OCP microscaling E8M0) -> 2^(e - 127) as a bf16x2
+// pair: the byte is the bf16 exponent field, except e = 0 (2^-127, a bf16
+// subnormal) and e = 255 (E8M0 NaN; reads as infinity here).
+__device__ __forceinline__ uint32_t ue8m0_bf16x2(uint32_t e) {
+  const uint32_t h = e ? (e << 7) : 0x40u;
+  return h | (h << 16);
+}
 
 // ---- tcgen05 (5th-generation tensor cores, tensor memory)
 __device__ __forceinline__ void tmem_alloc(uint32_t holder_smem, uint32_t ncols) {
@@ -425,12 +452,15 @@ __device__ __forceinline__ void tmem_st_16x32bx2_x32_h256(uint32_t taddr, const 
 // 16 lanes x 16 columns, twice: threads 0-15 write columns [c, c+16) of
 // lanes base+0..15, threads 16-31 columns [c+144, c+160) (the query's second
 // 288 dims).
+// kSplit: column offset of the second half (lanes 16-31 of the warp)
+template <int kSplit>
 __device__ __forceinline__ void tmem_st_16x32bx2_x16(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 144, "
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %17, "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+      "n"(kSplit)
       : "memory");
 }
 
@@ -570,10 +600,14 @@ __device__ __forceinline__ void merge_columns(const uint4* src, int d0, const fl
   }
 }
 
-template <bool kFp8>
-__global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
+template <int kKind>
+__global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     smla_split_kernel(const __grid_constant__ SplitParams p) {
-  constexpr int kCopy = Cfg<kFp8>::kCopyThreads;
+  constexpr int kCopy = Cfg<kKind>::kCopyThreads;
+  constexpr bool kFp8 = kKind == kKindFp8;     // row scale folded into S and P
+  constexpr bool kDsv4 = kKind == kKindDsv4;
+  constexpr bool kConv = Cfg<kKind>::kConv;
+  constexpr int kQK = kDsv4 ? 512 : kDqk;      // query / key width
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bars = sbase + kAuxBars;
@@ -599,6 +633,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 
   int* s_row = reinterpret_cast<int*>(smem + kAuxRow);
   float* s_rsc = reinterpret_cast<float*>(smem + kAuxRsc);
+  uint2* s_dsc = reinterpret_cast<uint2*>(smem + kAuxDsc);
 
   if (threadIdx.x == 0) {
     // Arrivals are per warp (the warp synchronises, one lane arrives), except
@@ -606,7 +641,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       // bf16: one arrival per copying thread (when its copies land); fp8:
       // one per convert warp
-      mbar_init(BAR(BAR_KVF + s), kFp8 ? Cfg<kFp8>::kCvtWarps : kCopy);
+      mbar_init(BAR(BAR_KVF + s), kConv ? Cfg<kKind>::kCvtWarps : kCopy);
       mbar_init(BAR(BAR_RAW + s), kCopy);
       mbar_init(BAR(BAR_KVE + s), 1);
       mbar_init(BAR(BAR_PF + s), 4);
@@ -625,7 +660,10 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     for (int r = 0; r < kRing; ++r) {
       mbar_init(BAR(BAR_IXF + r), 1);
       mbar_init(BAR(BAR_IXS + r), 1);
-      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + 4);
+      // consumers of a ring slot: the copy warps (rows), the softmax warps
+      // (row scales) and, for DeepSeek-V4 pages, the convert warps (scale
+      // blocks)
+      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + 4 + (kDsv4 ? Cfg<kKind>::kCvtWarps : 0));
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -657,19 +695,29 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       const int pos = tok_begin + t * kTile + j;
       return (t < ntiles && pos < tok_end) ? __ldg(p.indices + (size_t)b * p.topk + pos) : -1;
     };
+    // An entry that names no row of the pool (past the page table, or a
+    // row outside [0, num_kv_rows)) is read as padding and sets error bit 2.
     auto row_of = [&](int idx) -> int {
       if (idx < 0) return -1;
-      if (!p.page_size) return idx;
-      return __ldg(p.page_table + (size_t)b * p.pages_per_seq + idx / p.page_size) * p.page_size +
-             idx % p.page_size;
+      long long r = idx;
+      if (p.page_size) {
+        if (idx >= (long long)p.pages_per_seq * p.page_size) r = -1;
+        else r = (long long)__ldg(p.page_table + (size_t)b * p.pages_per_seq + idx / p.page_size) * p.page_size +
+                 idx % p.page_size;
+      }
+      if (r < 0 || r >= p.num_kv_rows) {
+        atomicOr(&g_error_word, 4u);
+        return -1;
+      }
+      return (int)r;
     };
     const int kw = warp - kWarpIdx;
-    // the 64 x 576 query (73,728 contiguous bytes) into the third KV stage,
-    // which no tile uses before the query has been moved to tensor memory
+    // the 64 x kQK query (contiguous bf16) into the third KV stage, which
+    // no tile uses before the query has been moved to tensor memory
     if (kw == 0 && lane == 0) {
-      mbar_arrive_expect_tx(BAR(BAR_QS), (uint32_t)kTileBytes);
-      bulk_load_g2s(sbase + kSmemKV + 2 * kTileBytes, p.q + (size_t)b * kH * kRowBytesBf16, (uint32_t)kTileBytes,
-                    BAR(BAR_QS));
+      constexpr uint32_t kQBytes = (uint32_t)kH * kQK * 2;
+      mbar_arrive_expect_tx(BAR(BAR_QS), kQBytes);
+      bulk_load_g2s(sbase + kSmemKV + 2 * kTileBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
     }
     // Software pipeline over this warp's tiles (step S = 4), every load
     // consumed one iteration after it was issued: index of tile t+3S, page
@@ -679,16 +727,32 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     int r1_0 = row_of(idx_at(kw + S, lane)), r1_1 = row_of(idx_at(kw + S, lane + 32));         // tile t+S
     int r0_0 = row_of(idx_at(kw, lane)), r0_1 = row_of(idx_at(kw, lane + 32));                 // tile t
     float c0_0 = 0.f, c0_1 = 0.f;                                            // scale, tile t
+    uint2 d0_0 = make_uint2(0u, 0u), d0_1 = make_uint2(0u, 0u);              // scale block, tile t
+    // a DeepSeek-V4 row's 8-byte scale block
+    auto dsc_of = [&](int r) -> uint2 {
+      if (r < 0) return make_uint2(0u, 0u);
+      return __ldg(reinterpret_cast<const uint2*>(p.kv + (size_t)(r >> 6) * kDsv4Page + kDsv4ScaleOff +
+                                                  (r & 63) * 8));
+    };
     if (kFp8) {
       c0_0 = r0_0 >= 0 ? __ldg(p.kv_row_scale + r0_0) : 0.f;
       c0_1 = r0_1 >= 0 ? __ldg(p.kv_row_scale + r0_1) : 0.f;
     }
+    if (kDsv4) {
+      d0_0 = dsc_of(r0_0);
+      d0_1 = dsc_of(r0_1);
+    }
     for (int t = kw; t < ntiles; t += S) {
       const int rs = t % kRing;
       float c1_0 = 0.f, c1_1 = 0.f;
+      uint2 d1_0 = make_uint2(0u, 0u), d1_1 = make_uint2(0u, 0u);
       if (kFp8) {
         c1_0 = r1_0 >= 0 ? __ldg(p.kv_row_scale + r1_0) : 0.f;
         c1_1 = r1_1 >= 0 ? __ldg(p.kv_row_scale + r1_1) : 0.f;
+      }
+      if (kDsv4) {
+        d1_0 = dsc_of(r1_0);
+        d1_1 = dsc_of(r1_1);
       }
       const int r2_0 = row_of(i2_0), r2_1 = row_of(i2_1);
       const int i3_0 = idx_at(t + 3 * S, lane), i3_1 = idx_at(t + 3 * S, lane + 32);
@@ -703,40 +767,64 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         s_rsc[rs * 64 + lane] = c0_0;
         s_rsc[rs * 64 + lane + 32] = c0_1;
       }
+      if (kDsv4) {
+        s_dsc[rs * 64 + lane] = d0_0;
+        s_dsc[rs * 64 + lane + 32] = d0_1;
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXS + rs));
       if (lane == 0 && t < 4) SMLA_TRACE_EV(58 + t);
       r0_0 = r1_0; r0_1 = r1_1;
       c0_0 = c1_0; c0_1 = c1_1;
+      d0_0 = d1_0; d0_1 = d1_1;
       r1_0 = r2_0; r1_1 = r2_1;
       i2_0 = i3_0; i2_1 = i3_1;
     }
-  } else if (warp >= kWarpLoad0 + Cfg<kFp8>::kCopyWarps) {
+  } else if (warp >= kWarpLoad0 + Cfg<kKind>::kCopyWarps) {
     // ------------------------------------------------- fp8 convert warps
     // Thread (tok, sub) turns the 16 codes of dims [16 sub, 16 sub + 16) of
     // every atom into bf16.  The copy warps put those codes in the first of
     // the two 16-byte chunks their bf16 values occupy in the swizzled tile,
     // so each thread reads and rewrites only its own two chunks: the
     // conversion runs in place with no barrier between threads.
-    const int ct = threadIdx.x - 32 * (kWarpLoad0 + Cfg<kFp8>::kCopyWarps);  // 0 .. 255
+    const int ct = threadIdx.x - 32 * (kWarpLoad0 + Cfg<kKind>::kCopyWarps);  // 0 .. 255
+    // DeepSeek-V4 pages: atoms 0..6 hold codes (times the group's UE8M0
+    // scale), atom 7 the bf16 rope dims, copied as they are
     const int tok = ct >> 2, sub = ct & 3;
+    constexpr int kCvtAtoms = kDsv4 ? kDsv4Nope / 64 : kAtoms;
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages;
+      uint2 dsc = make_uint2(0u, 0u);
+      if constexpr (kDsv4) {
+        const int rs = t % kRing;
+        if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXS + rs), (t / kRing) & 1))) break;
+        dsc = s_dsc[rs * 64 + tok];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
+      }
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + stage), (t / kStages) & 1))) break;
       if (ct == 0 && t < 8) SMLA_TRACE_EV(40 + t);
       const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
       const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
-      // all nine loads first (independent), then convert and store
-      uint4 v[kAtoms];
+      // all loads first (independent), then convert and store
+      uint4 v[kCvtAtoms];
 #pragma unroll
-      for (int a = 0; a < kAtoms; ++a) v[a] = ld_shared_v4(tbase + a * kAtomBytes + lo_off);
+      for (int a = 0; a < kCvtAtoms; ++a) v[a] = ld_shared_v4(tbase + a * kAtomBytes + lo_off);
 #pragma unroll
-      for (int a = 0; a < kAtoms; ++a) {
+      for (int a = 0; a < kCvtAtoms; ++a) {
         uint4 lo, hi;
-        e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
-        e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
-        e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
-        e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
+        if constexpr (kDsv4) {
+          const uint32_t s2 = ue8m0_bf16x2(((a < 4 ? dsc.x : dsc.y) >> (8 * (a & 3))) & 0xFFu);
+          e4m3x4_to_bf16x4_scaled(v[a].x, s2, lo.x, lo.y);
+          e4m3x4_to_bf16x4_scaled(v[a].y, s2, lo.z, lo.w);
+          e4m3x4_to_bf16x4_scaled(v[a].z, s2, hi.x, hi.y);
+          e4m3x4_to_bf16x4_scaled(v[a].w, s2, hi.z, hi.w);
+        } else {
+          e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
+          e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
+          e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
+          e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
+        }
         st_shared_v4(tbase + a * kAtomBytes + lo_off, lo);
         st_shared_v4(tbase + a * kAtomBytes + hi_off, hi);
       }
@@ -758,7 +846,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
       // 128-byte atom row; fp8: tokens 8(4 lw + u) + lane/4, 16 codes
       // (chunk lane%4) of a 64-byte atom row
       int rows[16];
-      if constexpr (!kFp8) {
+      if constexpr (!kConv) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) rows[u] = s_row[rs * 64 + 4 * u + (lane >> 3)];
       } else {
@@ -771,7 +859,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         break;
       // stage 2 first holds the staged query
       if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
-      if constexpr (!kFp8) {
+      if constexpr (!kConv) {
         if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
         // warp w copies atoms w, w+4, w+8; each warp instruction covers four
         // whole 128-byte row segments (coalesced); padding rows are
@@ -792,19 +880,34 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         if (lt == 0 && t < 8) SMLA_TRACE_EV(48 + t);
         // each warp instruction covers four whole 128-byte row segments
         // (a row is 4.5 segments); 16-code chunk c of a row goes to the first
-        // chunk of its bf16 destination (atom c / 4, see the convert warps)
+        // chunk of its bf16 destination (atom c / 4, see the convert warps).
+        // A DeepSeek-V4 slot is also 576 bytes: chunks 0..27 are codes, and
+        // the 64 bf16 rope dims (bytes 448..575) go straight to atom 7, lane
+        // j of a row's eight lanes copying rope chunk j.
         const int j = lane & 7;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int tok = 4 * (8 * lw + u) + (lane >> 3);
           const int row = rows[u];
-          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8;
+          const int rr = row >= 0 ? row : 0;
+          const uint32_t nbytes = row >= 0 ? 16u : 0u;
+          if constexpr (kDsv4) {
+            const uint8_t* src = p.kv + (size_t)(rr >> 6) * kDsv4Page + (rr & 63) * kDsv4Slot;
 #pragma unroll
-          for (int sg = 0; sg < 5; ++sg) {
-            const int c = 8 * sg + j;
-            if (c < kRowBytesFp8 / 16)
-              cp_async_16(tbase + (c >> 2) * kAtomBytes + sw128_off(tok, 2 * (c & 3)), src + c * 16,
-                          row >= 0 ? 16u : 0u);
+            for (int sg = 0; sg < 4; ++sg) {
+              const int c = 8 * sg + j;
+              if (c < kDsv4Nope / 16)
+                cp_async_16(tbase + (c >> 2) * kAtomBytes + sw128_off(tok, 2 * (c & 3)), src + c * 16, nbytes);
+            }
+            cp_async_16(tbase + 7 * kAtomBytes + sw128_off(tok, j), src + kDsv4Nope + j * 16, nbytes);
+          } else {
+            const uint8_t* src = p.kv + (size_t)rr * kRowBytesFp8;
+#pragma unroll
+            for (int sg = 0; sg < 5; ++sg) {
+              const int c = 8 * sg + j;
+              if (c < kRowBytesFp8 / 16)
+                cp_async_16(tbase + (c >> 2) * kAtomBytes + sw128_off(tok, 2 * (c & 3)), src + c * 16, nbytes);
+            }
           }
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_RAW + stage));
@@ -850,7 +953,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
         // +512, 16-element step +2
         mma_ts_set_elect(d, tmem + kColQ, bk, kIdescS);
 #pragma unroll
-        for (int k = 1; k < kDqk / 16; ++k) {
+        for (int k = 1; k < kQK / 16; ++k) {
           const uint64_t off = (uint64_t)((k >> 2) * (kAtomBytes >> 4) + (k & 3) * 2);
           mma_ts_acc_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + off, kIdescS);
         }
@@ -902,20 +1005,20 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     const int half = lane >> 4;
     const uint32_t q_lanes = (uint32_t)(32 * warp) << 16;            // Q / S rows
     const uint32_t o_lanes = (uint32_t)(32 * warp + kLaneO) << 16;   // O rows
-    {  // the query row into tensor memory: dims [288 half, 288 half + 288),
-       // read from the copy staged in shared memory (row-major [64][576])
+    {  // the query row into tensor memory: dims [kQK/2 half, +kQK/2), read
+       // from the copy staged in shared memory (row-major [64][kQK])
       bool okq = mbar_wait(BAR(BAR_QS), 0);
       if (okq) {
-        const uint8_t* qrow = smem + kSmemKV + 2 * kTileBytes + h * kRowBytesBf16 + half * 576;
+        const uint8_t* qrow = smem + kSmemKV + 2 * kTileBytes + h * (kQK * 2) + half * kQK;
 #pragma unroll 1
-        for (int c = 0; c < 9; ++c) {
+        for (int c = 0; c < kQK / 64; ++c) {
           uint32_t r[16];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint4 v = *reinterpret_cast<const uint4*>(qrow + c * 64 + u * 16);
             r[4 * u] = v.x; r[4 * u + 1] = v.y; r[4 * u + 2] = v.z; r[4 * u + 3] = v.w;
           }
-          tmem_st_16x32bx2_x16(tmem + q_lanes + kColQ + 16u * (uint32_t)c, r);  // second half at +144
+          tmem_st_16x32bx2_x16<kQK / 4>(tmem + q_lanes + kColQ + 16u * (uint32_t)c, r);  // second half at +kQK/4
         }
         tmem_wait_st();
       }
@@ -1282,9 +1385,14 @@ static smla_status validate_shape(const smla_shape* s) {
   if (s->batch < 1 || s->batch > 65535 || s->topk < 1 || s->topk > (1 << 24)) return SMLA_ERR_INVALID_ARG;
   if (s->num_kv_rows < 1 || s->num_kv_rows > 0x7FFFFFFFLL) return SMLA_ERR_INVALID_ARG;
   if (s->nsplit < 0 || s->reserved != 0) return SMLA_ERR_INVALID_ARG;
-  if (s->num_heads != kH || s->d_qk != kDqk || s->d_v != kDv) return SMLA_ERR_UNSUPPORTED;
-  if (s->kv_dtype != SMLA_KV_BF16 && s->kv_dtype != SMLA_KV_FP8_E4M3_ROWSCALE) return SMLA_ERR_UNSUPPORTED;
+  if (s->kv_dtype != SMLA_KV_BF16 && s->kv_dtype != SMLA_KV_FP8_E4M3_ROWSCALE && s->kv_dtype != SMLA_KV_DSV4_PAGED)
+    return SMLA_ERR_UNSUPPORTED;
+  const int want_qk = s->kv_dtype == SMLA_KV_DSV4_PAGED ? 512 : kDqk;
+  if (s->num_heads != kH || s->d_qk != want_qk || s->d_v != kDv) return SMLA_ERR_UNSUPPORTED;
   if (s->page_size != 0 && s->page_size != 64) return SMLA_ERR_UNSUPPORTED;
+  // DeepSeek-V4 pages hold 64 token slots: paged only, whole pages
+  if (s->kv_dtype == SMLA_KV_DSV4_PAGED && (s->page_size != 64 || s->num_kv_rows % 64 != 0))
+    return SMLA_ERR_UNSUPPORTED;
   if (s->page_size != 0 && s->pages_per_seq < 1) return SMLA_ERR_INVALID_ARG;
   return SMLA_OK;
 }
@@ -1363,14 +1471,14 @@ static size_t workspace_bytes_for(int batch, int nsplit, bool cluster) {
 // The shared-memory opt-in is set once per device (an idempotent call, so a
 // race between threads is harmless); later calls, including calls made
 // while a stream is being captured into a CUDA graph, skip it.
-template <bool kFp8>
+template <int kKind>
 static cudaError_t ensure_smem_attr() {
   static volatile int done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
   const cudaError_t e =
-      cudaFuncSetAttribute(smla_split_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      cudaFuncSetAttribute(smla_split_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
   return e;
 }
@@ -1381,7 +1489,7 @@ static cudaError_t ensure_smem_attr() {
 struct ClusterCaps {
   int active[5];  // index log2(c); active[0] unused
 };
-template <bool kFp8>
+template <int kKind>
 static const ClusterCaps& cluster_caps() {
   static ClusterCaps cache[64];
   static volatile int done[64] = {0};
@@ -1390,8 +1498,8 @@ static const ClusterCaps& cluster_caps() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return none;
   if (done[dev]) return cache[dev];
   ClusterCaps caps = {{0, 0, 0, 0, 0}};
-  if (ensure_smem_attr<kFp8>() == cudaSuccess &&
-      cudaFuncSetAttribute(smla_split_kernel<kFp8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+  if (ensure_smem_attr<kKind>() == cudaSuccess &&
+      cudaFuncSetAttribute(smla_split_kernel<kKind>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
     for (int lg = 1; lg <= 4; ++lg) {
       cudaLaunchAttribute at[1];
@@ -1401,12 +1509,12 @@ static const ClusterCaps& cluster_caps() {
       at[0].val.clusterDim.z = 1;
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(1u << lg, 1, 1);
-      cfg.blockDim = dim3(Cfg<kFp8>::kThreads, 1, 1);
+      cfg.blockDim = dim3(Cfg<kKind>::kThreads, 1, 1);
       cfg.dynamicSmemBytes = kSmemBytes;
       cfg.attrs = at;
       cfg.numAttrs = 1;
       int k = 0;
-      if (cudaOccupancyMaxActiveClusters(&k, smla_split_kernel<kFp8>, &cfg) == cudaSuccess) caps.active[lg] = k;
+      if (cudaOccupancyMaxActiveClusters(&k, smla_split_kernel<kKind>, &cfg) == cudaSuccess) caps.active[lg] = k;
     }
   }
   cudaGetLastError();  // a refused query leaves no sticky error
@@ -1415,13 +1523,15 @@ static const ClusterCaps& cluster_caps() {
   return cache[dev];
 }
 static const ClusterCaps& caps_for(const smla_shape* s) {
-  return s->kv_dtype == SMLA_KV_FP8_E4M3_ROWSCALE ? cluster_caps<true>() : cluster_caps<false>();
+  if (s->kv_dtype == SMLA_KV_FP8_E4M3_ROWSCALE) return cluster_caps<kKindFp8>();
+  if (s->kv_dtype == SMLA_KV_DSV4_PAGED) return cluster_caps<kKindDsv4>();
+  return cluster_caps<kKindBf16>();
 }
 
-template <bool kFp8>
+template <int kKind>
 static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
-  auto kern = smla_split_kernel<kFp8>;
-  cudaError_t e = ensure_smem_attr<kFp8>();
+  auto kern = smla_split_kernel<kKind>;
+  cudaError_t e = ensure_smem_attr<kKind>();
   if (e != cudaSuccess) return e;
   // programmatic dependent launch (the kernel waits for its prerequisites
   // itself), and for an in-cluster merge the cluster of nsplit CTAs
@@ -1439,7 +1549,7 @@ static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(prm.nsplit, prm.batch);
-  cfg.blockDim = dim3(Cfg<kFp8>::kThreads, 1, 1);
+  cfg.blockDim = dim3(Cfg<kKind>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = at;
@@ -1459,6 +1569,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
     return SMLA_ERR_INVALID_ARG;
   const bool fp8 = shape->kv_dtype == SMLA_KV_FP8_E4M3_ROWSCALE;
   if (fp8 && (!kv_row_scale || !aligned(kv_row_scale, 4))) return SMLA_ERR_INVALID_ARG;
+  if (shape->kv_dtype == SMLA_KV_DSV4_PAGED && kv_row_scale) return SMLA_ERR_INVALID_ARG;
   if (shape->page_size && (!page_table || !aligned(page_table, 4))) return SMLA_ERR_INVALID_ARG;
   if (!(scale == scale) || isinf(scale)) return SMLA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
@@ -1476,6 +1587,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.kv = static_cast<const uint8_t*>(kv_cache);
   prm.kv_row_scale = kv_row_scale;
   prm.page_table = page_table;
+  prm.num_kv_rows = (int)shape->num_kv_rows;
   prm.indices = indices;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
@@ -1491,7 +1603,9 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.page_size = shape->page_size;
   prm.pages_per_seq = shape->pages_per_seq;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
-  const cudaError_t e = fp8 ? launch_split<true>(prm, stream) : launch_split<false>(prm, stream);
+  const cudaError_t e = fp8 ? launch_split<kKindFp8>(prm, stream)
+                            : (shape->kv_dtype == SMLA_KV_DSV4_PAGED ? launch_split<kKindDsv4>(prm, stream)
+                                                                    : launch_split<kKindBf16>(prm, stream));
   if (e != cudaSuccess) return SMLA_ERR_CUDA;
   if (nsplit_out) *nsplit_out = n;
   if (nsplit_used) *nsplit_used = n;

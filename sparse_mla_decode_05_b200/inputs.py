@@ -223,7 +223,8 @@ def paged_dsv4(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: 
     perm = rng.permutation(total_pages)[: B * pps].reshape(B, pps)
     idx = np.stack([_distinct(rng, rows_per_seq, topk) for _ in range(B)])
     return Workload(name=name, q=q, kv=pages, indices=torch.from_numpy(idx.astype(np.int32)),
-                    page_table=torch.from_numpy(perm.astype(np.int32)), page_size=64, layout="dsv4",
+                    scale=1.0 / math.sqrt(512), page_table=torch.from_numpy(perm.astype(np.int32)),
+                    page_size=64, layout="dsv4",
                     meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages, topk=topk, seed=seed))
 
 
@@ -238,10 +239,17 @@ CONFIG_DESCRIPTIONS = {
     "c5": "B=128 k=2048 paged(64) fp8 e4m3 + row scale, 8192 rows/seq",
 }
 
+# Workloads beyond the headline set, measured and parity-tested the same way
+EXTRA_NAMES = ("dsv4",)
+EXTRA_DESCRIPTIONS = {
+    "dsv4": "B=32 k=512 DeepSeek-V4 pages (448 fp8 + UE8M0 group scales, 64 bf16 rope), 8192 rows/seq",
+}
+_BASE_SEEDS = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005, "dsv4": 1006}
+
 
 def make_config(name: str, seed: int | None = None) -> Workload:
-    """The full-size workload ``name`` (one of CONFIG_NAMES)."""
-    base = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005}[name]
+    """The full-size workload ``name`` (one of CONFIG_NAMES or EXTRA_NAMES)."""
+    base = _BASE_SEEDS[name]
     s = base if seed is None else seed
     if name == "c1":
         return flat_per_seq(1, 4096, 512, seed=s, name="c1")
@@ -255,6 +263,8 @@ def make_config(name: str, seed: int | None = None) -> Workload:
         return flat_per_seq(2, 65536, 2048, seed=s, q_mult=4.0, name="c4b")
     if name == "c5":
         return paged_fp8(128, 8192, 16384, 2048, seed=s, name="c5")
+    if name == "dsv4":
+        return paged_dsv4(32, 8192, 4096, 512, seed=s, name="dsv4")
     raise KeyError(name)
 
 
@@ -266,19 +276,23 @@ def shard_seed(name: str, rank: int) -> int | None:
         raise ValueError("rank must be >= 0")
     if rank == 0:
         return None
-    base = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005}[name]
-    return base + 100_000 * rank
+    return _BASE_SEEDS[name] + 100_000 * rank
 
 
 def algorithmic_bytes(w: Workload) -> int:
     """Bytes the step must move at minimum: valid gathered rows (row bytes,
-    plus the 4-byte row scale for fp8 pools), q, out, lse, the index list and
-    the page table.  Padding entries gather nothing."""
+    plus the 4-byte row scale for fp8 pools; a DeepSeek-V4 slot's 576 bytes
+    plus its 7 scale bytes), q, out, lse, the index list and the page
+    table.  Padding entries gather nothing."""
     n_valid = w.valid_count()
-    row = D_QK * (1 if w.kv.dtype == torch.uint8 else 2) + (4 if w.kv_row_scale is not None else 0)
+    if w.layout == "dsv4":
+        row, d_qk = 576 + 7, 512
+    else:
+        row = D_QK * (1 if w.kv.dtype == torch.uint8 else 2) + (4 if w.kv_row_scale is not None else 0)
+        d_qk = D_QK
     B = w.batch
     b = n_valid * row
-    b += B * H * D_QK * 2          # q
+    b += B * H * d_qk * 2          # q
     b += B * H * w.d_v * 2         # out
     b += B * H * 4                 # lse
     b += w.indices.numel() * 4     # indices
@@ -290,4 +304,4 @@ def algorithmic_bytes(w: Workload) -> int:
 def algorithmic_flops(w: Workload) -> int:
     """2*H*(d_qk + d_v) flops per valid (sequence, row): the score and the
     value contractions."""
-    return int(w.valid_count() * 2 * H * (D_QK + w.d_v))
+    return int(w.valid_count() * 2 * H * (w.q.shape[2] + w.d_v))

@@ -82,6 +82,9 @@ INVALID, UNSUPPORTED = 1, 2
     (dict(num_heads=32), UNSUPPORTED), (dict(d_qk=512), UNSUPPORTED), (dict(d_v=576), UNSUPPORTED),
     (dict(kv_dtype=7), UNSUPPORTED), (dict(page_size=32, pages_per_seq=4), UNSUPPORTED),
     (dict(page_size=64, pages_per_seq=0), INVALID),
+    # DeepSeek-V4 pages: d_qk 512, paged with 64-token pages, whole pages
+    (dict(kv_dtype=2), UNSUPPORTED), (dict(kv_dtype=2, d_qk=512), UNSUPPORTED),
+    (dict(kv_dtype=2, d_qk=512, page_size=64, pages_per_seq=4, num_kv_rows=1000), UNSUPPORTED),
 ])
 def test_bad_shapes_rejected_without_cuda(kw, code):
     assert _decode(shape(**kw)) == code
@@ -136,3 +139,12 @@ def test_python_binding_rejects_cpu_tensors():
         api.decode(q, kv, idx, 0.04)
     with pytest.raises(ValueError):
         api.decode(q[:, :32], kv, idx, 0.04)
+
+
+def test_dsv4_shape_accepted_and_row_scale_rejected():
+    s = api.make_shape(2, 100, 64 * 16, dsv4=True, page_size=64, pages_per_seq=8)
+    assert s.d_qk == 512 and s.kv_dtype == api.KV_DSV4_PAGED
+    assert api.lib.sparse_mla_plan_merge(ctypes.byref(s)) >= 0
+    # the pages carry their own scales: a row-scale pointer is an error,
+    # found before any CUDA call
+    assert _decode(s, rs=16, pt=16) == INVALID

@@ -397,3 +397,51 @@ def test_workspace_checks():
     one = a.shape_for(d.q, d.kv, d.indices, nsplit=1)
     assert a.workspace_size(one) == 0
     d.run(nsplit=1, workspace=None)                  # no workspace needed
+
+
+# ------------------------------------------------ entries naming no row
+@pytest.mark.parametrize("kind", ["flat_bf16", "paged_fp8", "dsv4"])
+def test_out_of_range_entries_read_as_padding(kind):
+    """An index past the pool (flat), past the page table's width (paged),
+    or resolving through a page-table entry outside the pool, is read as
+    padding and sets bit 2 of the device error word: the result equals the
+    oracle's with those entries replaced by -1."""
+    if kind == "flat_bf16":
+        w = inputs.flat_per_seq(3, 700, 300, seed=91)
+        n_rows = w.kv.shape[0]
+        bad = [n_rows, n_rows + 12345, 2 ** 31 - 1]
+    elif kind == "paged_fp8":
+        w = inputs.paged_fp8(3, 1024, 96, 300, seed=92)
+        bad = [1024, 1024 + 63, 2 ** 31 - 1]
+    else:
+        w = inputs.paged_dsv4(3, 1024, 96, 300, seed=93)
+        bad = [1024, 5000, 2 ** 31 - 1]
+    idx = w.indices.clone()
+    idx[0, 5] = bad[0]
+    idx[1, 100] = bad[1]
+    idx[2, 299] = bad[2]
+    clean = idx.clone()
+    clean[0, 5] = clean[1, 100] = clean[2, 299] = -1
+    if w.page_table is not None:
+        # a page-table entry that points past the pool
+        pt = w.page_table.clone()
+        pt[1, 0] = 96 + 5
+        pt[2, 1] = -3
+        hit = (idx >= 0) & (idx < 1024) & (((idx // 64 == 0) & (torch.arange(3)[:, None] == 1)) |
+                                            ((idx // 64 == 1) & (torch.arange(3)[:, None] == 2)))
+        clean[hit] = -1
+        w = inputs.Workload(name=w.name, q=w.q, kv=w.kv, indices=idx, scale=w.scale,
+                            kv_row_scale=w.kv_row_scale, page_table=pt, page_size=w.page_size,
+                            layout=w.layout)
+    else:
+        w = inputs.Workload(name=w.name, q=w.q, kv=w.kv, indices=idx, scale=w.scale)
+    w_clean = inputs.Workload(name=w.name, q=w.q, kv=w.kv, indices=clean, scale=w.scale,
+                              kv_row_scale=w.kv_row_scale, page_table=w.page_table,
+                              page_size=w.page_size, layout=w.layout)
+    d = Dev(w)
+    for n in (0, 1):
+        out, lse = d.run(nsplit=n)
+        torch.cuda.synchronize()
+        assert api().device_error() == 4
+        out_ref, lse_ref = oracle(w_clean)
+        assert_parity(out, lse, out_ref, lse_ref, tag=f"{kind} out-of-range n={n}")
