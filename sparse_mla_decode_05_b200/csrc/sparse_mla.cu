@@ -142,6 +142,8 @@ constexpr long long kWaitLimitCycles = 4000000000ll;
 // codes: two warps), then, for fp8 only, eight warps that convert the codes
 // to bf16 in place
 constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kIdxWarps = 4, kWarpLoad0 = kWarpIdx + kIdxWarps;
+// the in-cluster merge uses warps 0-7 and, for the lse, index warps 8-9
+static_assert(kWarpIdx <= 8 && kWarpIdx + kIdxWarps >= 10, "warps 8 and 9 must be index warps");
 // cache layouts the split kernel is instantiated for
 constexpr int kKindBf16 = 0;   // bf16 rows [N, 576]
 constexpr int kKindFp8 = 1;    // e4m3fn rows [N, 576] + one fp32 scale per row
@@ -562,23 +564,53 @@ __device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, u
                : "memory");
 }
 
-// In-cluster merge, final step for one thread: columns [d0, d0 + 64 / N * 4)
-// of one head (d0 = dim within its 256-dim half) from the N splits' fp16
-// images at src (one 16-byte unit = 8 dims; unit u of the half lives at
-// ((u / 4) * 4 + u % 4) * 32 lanes), weighted by w[s], times inv, to bf16.
+// In-cluster merge, final step for one thread: head hh, output columns
+// [col0, col0 + 128 / N) (16 / N units of 8 dims).  Split s's fp16 image
+// holds the thread's dims at lane hh % 16 (+16 for dims >= 256) of quarter
+// q, unit u of the half at ((u / 4) * 4 + u % 4) * 32 lanes.  Every split's
+// columns and statistics (m, l_pv) are loaded together, one L2 round trip
+// (with 16 splits the columns follow the weights), then split s is weighted
+// by 2^(m_s - M) l_pv,s and the sum divided by the sum of those weights.
 template <int N>
-__device__ __forceinline__ void merge_columns(const uint4* src, int d0, const float* w, float inv,
-                                              __nv_bfloat16* orow) {
+__device__ __forceinline__ void merge_tail(const float* wss, const uint4* wso, int q, int lane, int hh, int col0,
+                                           __nv_bfloat16* orow) {
   constexpr int kU = 16 / N;                     // units per split (16 loads in all)
   constexpr size_t kSplitU = (size_t)kH * kDv / 8;
+  const uint4* src = wso + (size_t)q * (8 * 4 * 32) + (lane & 15) + 16 * (col0 >> 8);
+  const int d0 = col0 & 255;
   uint4 x[16];
+  auto load_columns = [&]() {
 #pragma unroll
-  for (int s = 0; s < N; ++s)
+    for (int s = 0; s < N; ++s)
 #pragma unroll
-    for (int k = 0; k < kU; ++k) {
-      const int d = d0 + 8 * k;
-      x[s * kU + k] = __ldcg(src + (size_t)s * kSplitU + (size_t)((d >> 5) * 4 + ((d >> 3) & 3)) * 32);
-    }
+      for (int k = 0; k < kU; ++k) {
+        const int d = d0 + 8 * k;
+        x[s * kU + k] = __ldcg(src + (size_t)s * kSplitU + (size_t)((d >> 5) * 4 + ((d >> 3) & 3)) * 32);
+      }
+  };
+  // statistics [s][h] = (m, l_pv, l, -); the weights need m and l_pv
+  float w[N], lp[N];
+#pragma unroll
+  for (int s = 0; s < N; ++s) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(wss + ((size_t)s * 64 + hh) * 4));
+    w[s] = v.x; lp[s] = v.y;
+  }
+  // with 16 splits the columns are loaded after the weights (registers)
+  if constexpr (N < 16) load_columns();
+  float M = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < N; ++s) M = fmaxf(M, w[s]);
+  float Lp = 0.f;
+#pragma unroll
+  for (int s = 0; s < N; ++s) {
+    w[s] = (w[s] > -INFINITY ? ex2(w[s] - M) : 0.f) * lp[s];   // the weight of split s's normalised result
+    Lp += w[s];
+  }
+  const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
+  if constexpr (N >= 16) {
+    asm volatile("" ::: "memory");
+    load_columns();
+  }
 #pragma unroll
   for (int k = 0; k < kU; ++k) {
     float a[8];
@@ -1145,7 +1177,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       if (!aborted && half == 0) {
         float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
-        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4) = make_float4(m_run, l_tot, l_nrm, 0.f);
+        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4) = make_float4(m_run, l_nrm, l_tot, 0.f);
         // for the merge writers: 1 / (rounded-P sum) of head h
         reinterpret_cast<float*>(smem + kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
       }
@@ -1240,8 +1272,10 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // every PV has completed (the PV issuer's drain barrier: one phase)
       failed = !mbar_wait(BAR(BAR_FIN2), 0);
       tc_fence_after();
+      if (lane == 0 && warp == 4) SMLA_TRACE_EV(52);
     }
     const bool bad = group_any(failed, 1, 256);
+    if (threadIdx.x == 0) SMLA_TRACE_EV(48);
     if (!bad) {
       // this split's result for the thread's head, normalised by its own
       // rounded-P sum (a convex combination of value rows) and rounded to
@@ -1271,10 +1305,17 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         if (ntiles > 0 && cc + 1 < 4) tmem_wait_ld();
       }
     }
+    if (threadIdx.x == 0) SMLA_TRACE_EV(49);
     named_bar_sync(1, 256);
-    if (threadIdx.x == 0) {
-      fence_acq_rel_cluster();
-      for (int r = 0; r < n; ++r) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)r));
+    if (threadIdx.x == 0) SMLA_TRACE_EV(50);
+    // lane r of warp 0 arrives on CTA r's barrier: the n remote arrivals go
+    // out together (one after another they cost a round trip each)
+    if (warp == 0) {
+      if (lane == 0) fence_acq_rel_cluster();
+      __syncwarp();
+      if (lane == 0) SMLA_TRACE_EV(51);
+      if (lane < n) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)lane));
+      __syncwarp();
     }
     if (threadIdx.x == 0) SMLA_TRACE_EV(4);
     const bool ok = mbar_wait_cluster(BAR(BAR_CS1), 0);
@@ -1282,48 +1323,45 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     if (!group_any(bad || !ok, 1, 256)) {
       const int hh = 16 * q + (lane & 15);
       const int part = (lane >> 4) + 2 * upper;
-      float mv[16], lr[16], lp[16];
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        if (s2 < n) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
-          mv[s2] = v.x; lr[s2] = v.y; lp[s2] = v.z;
-        }
-      }
-      float M = -INFINITY;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2)
-        if (s2 < n) M = fmaxf(M, mv[s2]);
-      float Lr = 0.f, Lp = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        if (s2 < n) {
-          const float e = mv[s2] > -INFINITY ? ex2(mv[s2] - M) : 0.f;
-          Lr += e * lr[s2];
-          Lp += e * lp[s2];
-          mv[s2] = e * lp[s2];             // from here on: the weight of split s2's normalised result
-        }
-      }
-      const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
-      if (split == 0 && part == 0)
-        p.lse[(size_t)b * kH + hh] = Lr > 0.f ? (M + log2f(Lr)) * 0.6931471805599453f : -INFINITY;
-      if (threadIdx.x == 0) SMLA_TRACE_EV(56);
-      // this thread: columns [col0, col0 + cn / 4), 8 per 16-byte unit,
-      // stored by lane hh % 16 (+16 for dims >= 256) of quarter q
-      const int cn = kDv / n;
+      const int cn = kDv / n;                 // columns this CTA reduces
       const int col0 = split * cn + part * (cn / 4);
-      const uint4* src = wso + (size_t)q * (8 * 4 * 32) + (lane & 15) + 16 * (col0 >> 8);
       __nv_bfloat16* orow = p.out + ((size_t)b * kH + hh) * kDv + col0;
-      switch (n) {   // 16 loads per thread for every n: all issued before any is used
-        case 2: merge_columns<2>(src, col0 & 255, mv, inv, orow); break;
-        case 4: merge_columns<4>(src, col0 & 255, mv, inv, orow); break;
-        case 8: merge_columns<8>(src, col0 & 255, mv, inv, orow); break;
-        default: merge_columns<16>(src, col0 & 255, mv, inv, orow); break;
+      switch (n) {
+        case 2: merge_tail<2>(wss, wso, q, lane, hh, col0, orow); break;
+        case 4: merge_tail<4>(wss, wso, q, lane, hh, col0, orow); break;
+        case 8: merge_tail<8>(wss, wso, q, lane, hh, col0, orow); break;
+        default: merge_tail<16>(wss, wso, q, lane, hh, col0, orow); break;
       }
       if (threadIdx.x == 0) SMLA_TRACE_EV(62);
     }
     if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     tc_fence_before();
+  } else if (p.cluster && split == 0 && warp >= 8 && warp < 10) {
+    // lse of the merged result, head 32 (warp - 8) + lane, from every
+    // split's (m, l) once all have stored them: two index warps of rank 0,
+    // idle by now and outside the merging warps 0-7, alongside the column
+    // merge
+    const int hh = 32 * (warp - 8) + lane;
+    const float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
+    if (mbar_wait_cluster(BAR(BAR_CS1), 0)) {
+      float mv[16], lr[16];
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        mv[s2] = -INFINITY;
+        lr[s2] = 0.f;
+        if (s2 < p.nsplit) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
+          mv[s2] = v.x; lr[s2] = v.z;
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) M = fmaxf(M, mv[s2]);
+      float Lr = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) Lr += mv[s2] > -INFINITY ? ex2(mv[s2] - M) * lr[s2] : 0.f;
+      p.lse[(size_t)b * kH + hh] = Lr > 0.f ? (M + log2f(Lr)) * 0.6931471805599453f : -INFINITY;
+    }
   }
 
   __syncthreads();
