@@ -542,7 +542,6 @@ __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity) {
   }
   return true;
 }
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 // Programmatic dependent launch: the grid may start while the previous
 // kernel of the stream is still running (its prologue overlaps that
 // kernel's tail); griddepcontrol.wait blocks until every prerequisite grid
@@ -1310,9 +1309,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     if (threadIdx.x == 0) SMLA_TRACE_EV(50);
     // lane r of warp 0 arrives on CTA r's barrier: the n remote arrivals go
     // out together (one after another they cost a round trip each)
+    // (each arrival is a cluster-scope release: after the CTA barrier it
+    // covers every merging thread's stores)
     if (warp == 0) {
-      if (lane == 0) fence_acq_rel_cluster();
-      __syncwarp();
       if (lane == 0) SMLA_TRACE_EV(51);
       if (lane < n) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)lane));
       __syncwarp();
