@@ -243,6 +243,42 @@ smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void
                                              const int32_t* indices, float scale, void* out, float* lse,
                                              void* stream);
 
+/* Bytes of device staging that sparse_mla_decode_host needs for `shape`:
+ * q, indices, page table, out, lse and the decode workspace
+ * (sparse_mla_workspace_size), each region rounded up to 256 bytes, in that
+ * order.  Returns 0 for an invalid shape. */
+size_t sparse_mla_host_staging_size(const smla_shape* shape);
+
+/* The decode step with the per-step tensors in host memory; the cache
+ * (kv_cache, kv_row_scale) stays in device memory, where a serving engine
+ * keeps it.  The source pages have no counterpart to this entry point.
+ *
+ *   q_host, indices_host, page_table_host (when page_size > 0, else NULL):
+ *       host memory, laid out as for sparse_mla_decode
+ *   out_host [B, 64, 512] bf16, lse_host [B, 64] fp32: host memory, written
+ *   staging: device memory of >= sparse_mla_host_staging_size() bytes,
+ *       256-byte aligned, owned by the caller; contents need no
+ *       initialisation and are garbage afterwards
+ *
+ * On `stream`, in order: one cudaMemcpyAsync per input (host to device)
+ * into the staging, sparse_mla_decode on the staged copies, one
+ * cudaMemcpyAsync per result (device to host).  The call returns after
+ * enqueueing; the results are in out_host / lse_host once the stream has
+ * reached this point (synchronise the stream or an event).  Host buffers
+ * must be page-locked (cudaHostAlloc / cudaHostRegister) for the copies to
+ * be asynchronous; they must stay valid until then.  Calls that can
+ * overlap (different streams) need separate staging: two streams with one
+ * staging each overlap one step's copies with another step's decode.
+ *
+ * Errors: every argument is checked before the first copy is enqueued
+ * (SMLA_ERR_INVALID_ARG / SMLA_ERR_UNSUPPORTED as for sparse_mla_decode;
+ * SMLA_ERR_WORKSPACE for missing, misaligned or short staging);
+ * SMLA_ERR_CUDA if a copy or launch is refused. */
+smla_status sparse_mla_decode_host(const smla_shape* shape, const void* q_host, const void* kv_cache,
+                                   const float* kv_row_scale, const int32_t* page_table_host,
+                                   const int32_t* indices_host, float scale, void* out_host, float* lse_host,
+                                   void* staging, size_t staging_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,10 @@ def _load() -> ctypes.CDLL:
     lib.sparse_mla_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sparse_mla_decode_static_scratch.restype = I32
     lib.sparse_mla_decode_static_scratch.argtypes = [SP, P, P, P, P, P, F32, P, P, P]
+    lib.sparse_mla_host_staging_size.restype = SZ
+    lib.sparse_mla_host_staging_size.argtypes = [SP]
+    lib.sparse_mla_decode_host.restype = I32
+    lib.sparse_mla_decode_host.argtypes = [SP, P, P, P, P, P, F32, P, P, P, SZ, P]
     return lib
 
 
@@ -301,3 +305,91 @@ class DecodePlan:
         st = lib.sparse_mla_combine(*self._combine_args, self._stream if stream is None else stream)
         if st != 0:
             raise SmlaError(st, "sparse_mla_combine")
+
+
+# ------------------------------------------------- per-step tensors on the host
+def host_staging_size(shape: SmlaShape) -> int:
+    """Device staging bytes of sparse_mla_decode_host for ``shape``."""
+    return lib.sparse_mla_host_staging_size(ctypes.byref(shape))
+
+
+def _check_host_inputs(q_host, kv, indices_host, kv_row_scale, page_table_host, page_size, out_host, lse_host):
+    dsv4 = is_dsv4(kv)
+    d_qk = DSV4_D_QK if dsv4 else D_QK
+    for name, t in (("q_host", q_host), ("indices_host", indices_host), ("page_table_host", page_table_host),
+                    ("out_host", out_host), ("lse_host", lse_host)):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    for name, t in (("kv", kv), ("kv_row_scale", kv_row_scale)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if q_host.dtype != torch.bfloat16 or q_host.dim() != 3 or q_host.shape[1:] != (H, d_qk):
+        raise ValueError(f"q_host must be bf16 [B, 64, {d_qk}]")
+    B = q_host.shape[0]
+    if indices_host.dtype != torch.int32 or indices_host.dim() != 2 or indices_host.shape[0] != B:
+        raise ValueError("indices_host must be int32 [B, topk]")
+    if page_size and (page_table_host is None or page_table_host.dtype != torch.int32):
+        raise ValueError("paged cache needs int32 page_table_host [B, pages_per_seq]")
+    if out_host.dtype != torch.bfloat16 or tuple(out_host.shape) != (B, H, D_V):
+        raise ValueError("out_host must be bf16 [B, 64, 512]")
+    if lse_host.dtype != torch.float32 or tuple(lse_host.shape) != (B, H):
+        raise ValueError("lse_host must be float32 [B, 64]")
+
+
+class HostDecodePlan:
+    """sparse_mla_decode_host with its arguments marshalled once.
+
+    q_host, indices_host (and page_table_host) are host tensors the caller
+    refills between steps; out_host and lse_host receive each step's
+    results.  Pinned host tensors make the copies asynchronous.  kv and
+    kv_row_scale are device tensors.  run(stream) enqueues one step (copies
+    in, decode, copies out) on ``stream`` (default: the current stream) and
+    returns; the results are ready once that stream has reached it.  Plans
+    used on different streams at the same time need their own staging,
+    which each plan allocates unless one is given."""
+
+    def __init__(self, q_host, kv, indices_host, scale: float, *, kv_row_scale=None, page_table_host=None,
+                 page_size: int = 0, nsplit: int = 0, out_host=None, lse_host=None, staging=None):
+        B = q_host.shape[0]
+        pin = q_host.is_pinned()
+        if out_host is None:
+            out_host = torch.empty((B, H, D_V), dtype=torch.bfloat16, pin_memory=pin)
+        if lse_host is None:
+            lse_host = torch.empty((B, H), dtype=torch.float32, pin_memory=pin)
+        _check_host_inputs(q_host, kv, indices_host, kv_row_scale, page_table_host, page_size, out_host,
+                           lse_host)
+        if is_dsv4(kv):
+            if kv_row_scale is not None or page_size != 64:
+                raise ValueError("DeepSeek-V4 pages: no kv_row_scale, page_size 64")
+        elif (kv.dtype == torch.uint8) != (kv_row_scale is not None):
+            raise ValueError("an fp8 cache needs kv_row_scale, a bf16 cache none")
+        self.shape = shape_for(q_host, kv, indices_host, page_table=page_table_host, page_size=page_size,
+                               nsplit=nsplit)
+        need = host_staging_size(self.shape)
+        if staging is None:
+            staging = torch.empty(need, dtype=torch.uint8, device=kv.device)
+        self.out_host, self.lse_host, self.staging = out_host, lse_host, staging
+        self._keep = (q_host, kv, indices_host, kv_row_scale, page_table_host)
+        self._device = kv.device
+        self._args = (ctypes.byref(self.shape), _ptr(q_host), _ptr(kv), _ptr(kv_row_scale), _ptr(page_table_host),
+                      _ptr(indices_host), float(scale), _ptr(out_host), _ptr(lse_host), _ptr(staging),
+                      staging.numel())
+
+    def run(self, stream=None):
+        s = _stream(self._device) if stream is None else (stream.cuda_stream if hasattr(stream, "cuda_stream")
+                                                          else stream)
+        st = lib.sparse_mla_decode_host(*self._args, s)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_decode_host")
+
+
+def decode_host(q_host, kv, indices_host, scale: float, *, kv_row_scale=None, page_table_host=None,
+                page_size: int = 0, nsplit: int = 0, out_host=None, lse_host=None):
+    """One decode step with the per-step tensors on the host: returns
+    (out_host, lse_host) after synchronising the current stream."""
+    plan = HostDecodePlan(q_host, kv, indices_host, scale, kv_row_scale=kv_row_scale,
+                          page_table_host=page_table_host, page_size=page_size, nsplit=nsplit,
+                          out_host=out_host, lse_host=lse_host)
+    plan.run()
+    torch.cuda.current_stream(kv.device).synchronize()
+    return plan.out_host, plan.lse_host

@@ -1684,6 +1684,31 @@ static smla_status static_scratch_address(void** ptr) {
   return SMLA_OK;
 }
 
+// Device staging of sparse_mla_decode_host: q, indices, page table, out,
+// lse and the decode workspace, each region 256-byte aligned.
+struct HostStaging {
+  size_t q, q_bytes, idx, idx_bytes, pt, pt_bytes, out, out_bytes, lse, lse_bytes, ws, ws_bytes, total;
+};
+static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+static HostStaging host_staging(const smla_shape* s, size_t ws_bytes) {
+  HostStaging h;
+  size_t off = 0;
+  h.q_bytes = (size_t)s->batch * kH * s->d_qk * 2;
+  h.idx_bytes = (size_t)s->batch * s->topk * 4;
+  h.pt_bytes = s->page_size ? (size_t)s->batch * s->pages_per_seq * 4 : 0;
+  h.out_bytes = (size_t)s->batch * kH * kDv * 2;
+  h.lse_bytes = (size_t)s->batch * kH * 4;
+  h.ws_bytes = ws_bytes;
+  h.q = off;   off += round256(h.q_bytes);
+  h.idx = off; off += round256(h.idx_bytes);
+  h.pt = off;  off += round256(h.pt_bytes);
+  h.out = off; off += round256(h.out_bytes);
+  h.lse = off; off += round256(h.lse_bytes);
+  h.ws = off;  off += round256(h.ws_bytes);
+  h.total = off;
+  return h;
+}
+
 }  // namespace smla
 
 // ============================================================ C ABI
@@ -1785,6 +1810,48 @@ smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void
   fixed.nsplit = n;
   return sparse_mla_decode(&fixed, q, kv_cache, kv_row_scale, page_table, indices, scale, out, lse, scratch,
                            need, stream);
+}
+
+size_t sparse_mla_host_staging_size(const smla_shape* shape) {
+  if (smla::validate_shape(shape) != SMLA_OK) return 0;
+  return smla::host_staging(shape, sparse_mla_workspace_size(shape)).total;
+}
+
+smla_status sparse_mla_decode_host(const smla_shape* shape, const void* q_host, const void* kv_cache,
+                                   const float* kv_row_scale, const int32_t* page_table_host,
+                                   const int32_t* indices_host, float scale, void* out_host, float* lse_host,
+                                   void* staging, size_t staging_bytes, void* stream) {
+  smla_status st = smla::validate_shape(shape);
+  if (st != SMLA_OK) return st;
+  // every argument check before the first copy is enqueued
+  if (!q_host || !kv_cache || !indices_host || !out_host || !lse_host) return SMLA_ERR_INVALID_ARG;
+  if (!smla::aligned(kv_cache, 16)) return SMLA_ERR_INVALID_ARG;
+  if ((shape->page_size != 0) != (page_table_host != nullptr)) return SMLA_ERR_INVALID_ARG;
+  const bool fp8 = shape->kv_dtype == SMLA_KV_FP8_E4M3_ROWSCALE;
+  if (fp8 != (kv_row_scale != nullptr)) return SMLA_ERR_INVALID_ARG;
+  if (fp8 && !smla::aligned(kv_row_scale, 4)) return SMLA_ERR_INVALID_ARG;
+  if (!(scale == scale) || isinf(scale)) return SMLA_ERR_INVALID_ARG;
+  if (!staging || !smla::aligned(staging, 256)) return SMLA_ERR_WORKSPACE;
+  const size_t ws = sparse_mla_workspace_size(shape);
+  const smla::HostStaging h = smla::host_staging(shape, ws);
+  if (staging_bytes < h.total) return SMLA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(staging);
+  // one copy per tensor (host to device), the step, then the results back
+  if (cudaMemcpyAsync(base + h.q, q_host, h.q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(base + h.idx, indices_host, h.idx_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      (h.pt_bytes && cudaMemcpyAsync(base + h.pt, page_table_host, h.pt_bytes, cudaMemcpyHostToDevice, s) !=
+                         cudaSuccess))
+    return SMLA_ERR_CUDA;
+  st = sparse_mla_decode(shape, base + h.q, kv_cache, kv_row_scale,
+                         h.pt_bytes ? reinterpret_cast<const int32_t*>(base + h.pt) : nullptr,
+                         reinterpret_cast<const int32_t*>(base + h.idx), scale, base + h.out,
+                         reinterpret_cast<float*>(base + h.lse), ws ? base + h.ws : nullptr, ws, stream);
+  if (st != SMLA_OK) return st;
+  if (cudaMemcpyAsync(out_host, base + h.out, h.out_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(lse_host, base + h.lse, h.lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SMLA_ERR_CUDA;
+  return SMLA_OK;
 }
 
 smla_status sparse_mla_get_device_error(uint32_t* code) {

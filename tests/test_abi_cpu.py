@@ -148,3 +148,47 @@ def test_dsv4_shape_accepted_and_row_scale_rejected():
     # the pages carry their own scales: a row-scale pointer is an error,
     # found before any CUDA call
     assert _decode(s, rs=16, pt=16) == INVALID
+
+
+# ------------------------------------------------ sparse_mla_decode_host
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_host_staging_size_is_the_sum_of_its_regions():
+    # q, indices, page table, out, lse (workspace 0: one split without a device)
+    s = api.make_shape(16, 512, 67000)
+    assert api.host_staging_size(s) == (_r256(16 * 64 * 576 * 2) + _r256(16 * 512 * 4) + _r256(16 * 64 * 512 * 2)
+                                        + _r256(16 * 64 * 4))
+    s = api.make_shape(3, 100, 64 * 40, fp8=True, page_size=64, pages_per_seq=7)
+    assert api.host_staging_size(s) == (_r256(3 * 64 * 576 * 2) + _r256(3 * 100 * 4) + _r256(3 * 7 * 4)
+                                        + _r256(3 * 64 * 512 * 2) + _r256(3 * 64 * 4))
+    s = api.make_shape(2, 100, 64 * 16, dsv4=True, page_size=64, pages_per_seq=8)
+    assert api.host_staging_size(s) == (_r256(2 * 64 * 512 * 2) + _r256(2 * 100 * 4) + _r256(2 * 8 * 4)
+                                        + _r256(2 * 64 * 512 * 2) + _r256(2 * 64 * 4))
+    assert api.host_staging_size(shape(batch=0)) == 0
+
+
+def _host(s, q=16, kv=16, rs=None, pt=None, idx=16, scale=0.04, out=16, lse=16, st=256, nbytes=1 << 30):
+    return api.lib.sparse_mla_decode_host(ctypes.byref(s) if s is not None else None, q, kv, rs, pt, idx, scale,
+                                          out, lse, st, nbytes, None)
+
+
+WORKSPACE = 3
+
+
+def test_decode_host_rejects_bad_arguments_before_any_copy():
+    s = shape()
+    assert _host(None) == INVALID
+    assert _host(shape(batch=0)) == INVALID
+    for kw in (dict(q=None), dict(kv=None), dict(idx=None), dict(out=None), dict(lse=None)):
+        assert _host(s, **kw) == INVALID
+    assert _host(s, kv=8) == INVALID                     # cache not 16-byte aligned
+    assert _host(s, pt=16) == INVALID                    # page table without paging
+    assert _host(shape(page_size=64, pages_per_seq=4)) == INVALID   # paging without a page table
+    assert _host(s, rs=16) == INVALID                    # row scale with a bf16 cache
+    assert _host(shape(fp8=True)) == INVALID             # fp8 cache without row scales
+    assert _host(s, scale=float("nan")) == INVALID
+    assert _host(s, st=None) == WORKSPACE
+    assert _host(s, st=128) == WORKSPACE                 # staging not 256-byte aligned
+    assert _host(s, nbytes=api.host_staging_size(s) - 1) == WORKSPACE
