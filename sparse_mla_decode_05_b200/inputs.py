@@ -228,6 +228,60 @@ def paged_dsv4(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: 
                     meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages, topk=topk, seed=seed))
 
 
+@dataclasses.dataclass
+class IndexerWorkload:
+    """Inputs of the indexer step: the decode token's indexer query and head
+    weights per sequence, a paged bf16 key cache, page tables and context
+    lengths."""
+    name: str
+    q: torch.Tensor            # [B, H, D] bfloat16
+    w: torch.Tensor            # [B, H] float32
+    k: torch.Tensor            # [pages * 64, D] bfloat16
+    page_table: torch.Tensor   # [B, pages_per_seq] int32
+    ctx_len: torch.Tensor      # [B] int32
+    max_ctx: int
+    topk: int
+    meta: dict = dataclasses.field(default_factory=dict)
+
+    @property
+    def batch(self) -> int:
+        return self.q.shape[0]
+
+
+def indexer_workload(B: int, max_ctx: int, total_pages: int, *, seed: int, topk: int = 512, H: int = 64,
+                     D: int = 128, ctx_lo: int | None = None, name: str = "indexer") -> IndexerWorkload:
+    """Seeded indexer inputs: q and k N(0,1) in bf16, w N(0,1)/sqrt(H) in
+    fp32 (signed), context lengths uniform in [ctx_lo, max_ctx] (all equal to
+    max_ctx when ctx_lo is None), page tables slices of one random
+    permutation of all pages."""
+    pps = (max_ctx + 63) // 64
+    if B * pps > total_pages:
+        raise ValueError("not enough pages for distinct page tables")
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(gen, (B, H, D))
+    w = (torch.randn((B, H), generator=gen, dtype=torch.float32) / math.sqrt(H)).contiguous()
+    k = _normal_bf16(gen, (total_pages * 64, D))
+    perm = rng.permutation(total_pages)[: B * pps].reshape(B, pps)
+    if ctx_lo is None:
+        ctx = np.full(B, max_ctx)
+    else:
+        ctx = rng.integers(ctx_lo, max_ctx + 1, size=B)
+    return IndexerWorkload(name=name, q=q, w=w, k=k, page_table=torch.from_numpy(perm.astype(np.int32)),
+                           ctx_len=torch.from_numpy(ctx.astype(np.int32)), max_ctx=max_ctx, topk=topk,
+                           meta=dict(B=B, max_ctx=max_ctx, total_pages=total_pages, seed=seed, H=H, D=D))
+
+
+def indexer_algorithmic_bytes(w: IndexerWorkload) -> int:
+    """Bytes the indexer step must move at minimum: the keys of every
+    context position (D bf16 each), q, w, the page tables, the context
+    lengths and the selected index lists."""
+    D = w.q.shape[2]
+    n = int(w.ctx_len.sum())
+    return int(n * D * 2 + w.q.numel() * 2 + w.w.numel() * 4 + w.page_table.numel() * 4 + w.batch * 4
+               + w.batch * w.topk * 4)
+
+
 CONFIG_NAMES = ("c1", "c2", "c3", "c4a", "c4b", "c5")
 
 CONFIG_DESCRIPTIONS = {
