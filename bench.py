@@ -445,6 +445,25 @@ def main():
             if rc is not r:
                 del rc
                 torch.cuda.empty_cache()
+        # the indexer step that produces the index lists (scores + top-k)
+        wi = inputs.make_indexer_config()
+        ip = api.IndexerPlan(wi.q.to(dev), wi.w.to(dev), wi.k.to(dev), wi.page_table.to(dev),
+                             wi.ctx_len.to(dev), wi.topk, max_ctx=wi.max_ctx)
+        tms = time_device(ip.run, 30, 3, flush, stream)
+        med = float(np.median(tms)) * 1e3
+        ab = inputs.indexer_algorithmic_bytes(wi)
+        fl = 2 * wi.q.shape[1] * wi.q.shape[2] * int(wi.ctx_len.sum())
+        rl = max(ab / (peak_gbs * 1e3), fl / (peak_tf * 1e6))
+        per_config.append({"workload": "indexer", "description": inputs.INDEXER_DESCRIPTION, "batch": wi.batch,
+                           "topk": wi.topk, "max_ctx": wi.max_ctx, "us_per_call": med,
+                           "p10_us": float(np.percentile(tms, 10)) * 1e3,
+                           "p90_us": float(np.percentile(tms, 90)) * 1e3,
+                           "gbs": ab / (med * 1e-6) / 1e9, "roofline_us": rl, "frac_roofline": rl / med,
+                           "scores_kernel_us": float(np.median(time_device(ip.run_scores, 15, 3, flush, stream))) * 1e3,
+                           "topk_kernel_us": float(np.median(time_device(ip.run_topk, 15, 3, flush, stream))) * 1e3,
+                           "alg_bytes": ab, "alg_flops": fl})
+        del ip
+        torch.cuda.empty_cache()
         assert api.device_error() == 0, "device error word set"
 
     # --- CPU baseline: the oracle on host cores, bounded sample

@@ -279,6 +279,64 @@ smla_status sparse_mla_decode_host(const smla_shape* shape, const void* q_host, 
                                    const int32_t* indices_host, float scale, void* out_host, float* lse_host,
                                    void* staging, size_t staging_bytes, void* stream);
 
+/* ------------------------------------------------------------------ indexer
+ * The step upstream of the decode: it scores every position of each
+ * sequence's context and picks the top-k positions the decode attends to
+ * ("The Pivot Point: When a 6.3x Kernel Speedup Reveals the Next
+ * Bottleneck", "Input Knowledge Required": the indexer selects the top ~512
+ * cache positions per decode step; "The Context: A Campaign in Full Swing":
+ * its batched matrix product runs on bf16 tensor cores; "The Moment of
+ * Truth: Benchmarking a Custom MMA Kernel for DeepSeek-V4-Flash on
+ * Blackwell", "Broader Context": only the real context is scored).
+ *
+ * Scores, in the published form of DeepSeek's sparse-attention indexer (the
+ * pages name only the batched product and the top-k):
+ *   I[b, s] = sum_h w[b, h] * max(0, q[b, h, :] . k[row(b, s), :]),  s < ctx_len[b]
+ * accumulated in fp32 (each head's dot product on the tensor cores, the
+ * weighted sum over heads in order h = 0 .. 63), with
+ * row(b, s) = page_table[b, s / 64] * 64 + s % 64.
+ * Selection: the min(topk, ctx_len[b]) positions with the largest I[b, s],
+ * ties to the lower position, written in ascending order, then -1. */
+typedef struct {
+  int32_t batch;          /* B, 1 .. 65535                                     */
+  int32_t heads;          /* 64                                                */
+  int32_t dim;            /* 128 (bf16 per head)                               */
+  int32_t topk;           /* 1 .. 65536                                        */
+  int32_t max_ctx;        /* width of a score row: 1 .. 2^20, >= every ctx_len */
+  int32_t page_size;      /* 64                                                */
+  int32_t pages_per_seq;  /* page-table width; 64 * pages_per_seq >= max_ctx   */
+  int32_t reserved;       /* must be 0                                         */
+  int64_t num_key_rows;   /* rows in the key cache, a multiple of 64           */
+} smla_indexer_shape;
+
+/* Scores of every position (the indexer's batched product).
+ *   q         [B, 64, 128] bf16, 16-byte aligned
+ *   w         [B, 64] fp32 head weights
+ *   k_cache   [num_key_rows, 128] bf16 keys, 16-byte aligned (64-row pages)
+ *   page_table[B, pages_per_seq] int32, ctx_len [B] int32
+ *   scores    [B, max_ctx] fp32, written: I[b, s] for s < ctx_len[b], -inf
+ *             after (-0 is written as +0)
+ * All device memory, caller-owned.  A ctx_len outside [0, max_ctx] is
+ * clamped and a page-table entry outside the cache reads as absent keys;
+ * both set bit 2 of the device error word.  Returns after launching. */
+smla_status sparse_mla_indexer_scores(const smla_indexer_shape* shape, const void* q, const float* w,
+                                      const void* k_cache, const int32_t* page_table, const int32_t* ctx_len,
+                                      float* scores, void* stream);
+
+/* Top-k positions from a score matrix laid out as above:
+ *   indices [B, topk] int32, written (ascending positions, -1 padding).
+ * Reads scores[b, 0 .. ctx_len[b]) only; ctx_len as above. */
+smla_status sparse_mla_indexer_topk(const smla_indexer_shape* shape, const float* scores, const int32_t* ctx_len,
+                                    int32_t* indices, void* stream);
+
+/* Both steps: scores into the caller's `scores` buffer ([B, max_ctx] fp32,
+ * kept for inspection), then the top-k into `indices`.  Two launches on
+ * `stream`; the second may start its prologue early (programmatic
+ * dependent launch) and waits for the first. */
+smla_status sparse_mla_indexer(const smla_indexer_shape* shape, const void* q, const float* w, const void* k_cache,
+                               const int32_t* page_table, const int32_t* ctx_len, float* scores,
+                               int32_t* indices, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

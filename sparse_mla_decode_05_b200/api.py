@@ -38,6 +38,15 @@ class SmlaShape(ctypes.Structure):
     ]
 
 
+class IndexerShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("dim", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("max_ctx", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("pages_per_seq", ctypes.c_int32), ("reserved", ctypes.c_int32), ("num_key_rows", ctypes.c_int64)]
+
+
+IX_HEADS, IX_DIM = 64, 128
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -65,6 +74,13 @@ def _load() -> ctypes.CDLL:
     lib.sparse_mla_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sparse_mla_decode_static_scratch.restype = I32
     lib.sparse_mla_decode_static_scratch.argtypes = [SP, P, P, P, P, P, F32, P, P, P]
+    IP = ctypes.POINTER(IndexerShape)
+    lib.sparse_mla_indexer_scores.restype = I32
+    lib.sparse_mla_indexer_scores.argtypes = [IP, P, P, P, P, P, P, P]
+    lib.sparse_mla_indexer_topk.restype = I32
+    lib.sparse_mla_indexer_topk.argtypes = [IP, P, P, P, P]
+    lib.sparse_mla_indexer.restype = I32
+    lib.sparse_mla_indexer.argtypes = [IP, P, P, P, P, P, P, P, P]
     lib.sparse_mla_host_staging_size.restype = SZ
     lib.sparse_mla_host_staging_size.argtypes = [SP]
     lib.sparse_mla_decode_host.restype = I32
@@ -393,3 +409,71 @@ def decode_host(q_host, kv, indices_host, scale: float, *, kv_row_scale=None, pa
     plan.run()
     torch.cuda.current_stream(kv.device).synchronize()
     return plan.out_host, plan.lse_host
+
+
+# ------------------------------------------------------------------ indexer
+def indexer_shape(batch: int, topk: int, max_ctx: int, pages_per_seq: int, num_key_rows: int) -> IndexerShape:
+    return IndexerShape(batch, IX_HEADS, IX_DIM, topk, max_ctx, 64, pages_per_seq, 0, num_key_rows)
+
+
+def _check_indexer(q, w, k_cache, page_table, ctx_len):
+    for name, t in (("q", q), ("w", w), ("k_cache", k_cache), ("page_table", page_table), ("ctx_len", ctx_len)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[1:] != (IX_HEADS, IX_DIM):
+        raise ValueError("q must be bf16 [B, 64, 128]")
+    B = q.shape[0]
+    if w.dtype != torch.float32 or tuple(w.shape) != (B, IX_HEADS):
+        raise ValueError("w must be float32 [B, 64]")
+    if k_cache.dtype != torch.bfloat16 or k_cache.dim() != 2 or k_cache.shape[1] != IX_DIM:
+        raise ValueError("k_cache must be bf16 [rows, 128]")
+    if page_table.dtype != torch.int32 or page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be int32 [B, pages_per_seq]")
+    if ctx_len.dtype != torch.int32 or tuple(ctx_len.shape) != (B,):
+        raise ValueError("ctx_len must be int32 [B]")
+
+
+class IndexerPlan:
+    """The indexer step with its arguments marshalled once: scores
+    ([B, max_ctx] fp32) and the top-k positions ([B, topk] int32) into
+    buffers the plan owns (or the caller gives).  run() is one call into
+    the library (two launches)."""
+
+    def __init__(self, q, w, k_cache, page_table, ctx_len, topk: int, *, max_ctx: int | None = None,
+                 scores=None, indices=None):
+        _check_indexer(q, w, k_cache, page_table, ctx_len)
+        B = q.shape[0]
+        if max_ctx is None:
+            max_ctx = page_table.shape[1] * 64
+        self.shape = indexer_shape(B, topk, max_ctx, page_table.shape[1], k_cache.shape[0])
+        dev = q.device
+        self.scores = scores if scores is not None else torch.empty((B, max_ctx), dtype=torch.float32, device=dev)
+        self.indices = indices if indices is not None else torch.empty((B, topk), dtype=torch.int32, device=dev)
+        self._keep = (q, w, k_cache, page_table, ctx_len)
+        self._stream = _stream(dev)
+        self._args = (ctypes.byref(self.shape), _ptr(q), _ptr(w), _ptr(k_cache), _ptr(page_table), _ptr(ctx_len),
+                      _ptr(self.scores), _ptr(self.indices))
+
+    def run(self, stream=None):
+        st = lib.sparse_mla_indexer(*self._args, self._stream if stream is None else stream)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_indexer")
+
+    def run_scores(self, stream=None):
+        st = lib.sparse_mla_indexer_scores(*self._args[:7], self._stream if stream is None else stream)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_indexer_scores")
+
+    def run_topk(self, stream=None):
+        st = lib.sparse_mla_indexer_topk(self._args[0], self._args[6], self._args[5], self._args[7],
+                                         self._stream if stream is None else stream)
+        if st != 0:
+            raise SmlaError(st, "sparse_mla_indexer_topk")
+
+
+def indexer(q, w, k_cache, page_table, ctx_len, topk: int, *, max_ctx: int | None = None):
+    """One indexer step: returns (indices [B, topk] int32, scores [B, max_ctx]
+    fp32), enqueued on the current stream."""
+    plan = IndexerPlan(q, w, k_cache, page_table, ctx_len, topk, max_ctx=max_ctx)
+    plan.run()
+    return plan.indices, plan.scores

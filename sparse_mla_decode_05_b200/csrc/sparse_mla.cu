@@ -1711,6 +1711,9 @@ static HostStaging host_staging(const smla_shape* s, size_t ws_bytes) {
 
 }  // namespace smla
 
+// the indexer step (scores and top-k selection), sharing the helpers above
+#include "indexer.cuh"
+
 // ============================================================ C ABI
 extern "C" {
 

@@ -187,6 +187,24 @@ def paged_fp8(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: i
                               topk=topk, seed=seed))
 
 
+def paged_bf16(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: int,
+               name: str = "paged_bf16") -> Workload:
+    """Paged bf16 pool [total_pages * 64, 576] of N(0,1) rows; page tables
+    and index lists as in paged_fp8."""
+    pps = rows_per_seq // 64
+    if B * pps > total_pages:
+        raise ValueError("not enough pages for distinct page tables")
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(gen, (B, H, D_QK))
+    kv = _normal_bf16(gen, (total_pages * 64, D_QK))
+    perm = rng.permutation(total_pages)[: B * pps].reshape(B, pps)
+    idx = np.stack([_distinct(rng, rows_per_seq, topk) for _ in range(B)])
+    return Workload(name=name, q=q, kv=kv, indices=torch.from_numpy(idx.astype(np.int32)),
+                    page_table=torch.from_numpy(perm.astype(np.int32)), page_size=64,
+                    meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages, topk=topk, seed=seed))
+
+
 DSV4_PAGE_BYTES = 64 * 584          # 64 slots of 576 bytes, then 64 scale blocks of 8 bytes
 
 
@@ -270,6 +288,16 @@ def indexer_workload(B: int, max_ctx: int, total_pages: int, *, seed: int, topk:
     return IndexerWorkload(name=name, q=q, w=w, k=k, page_table=torch.from_numpy(perm.astype(np.int32)),
                            ctx_len=torch.from_numpy(ctx.astype(np.int32)), max_ctx=max_ctx, topk=topk,
                            meta=dict(B=B, max_ctx=max_ctx, total_pages=total_pages, seed=seed, H=H, D=D))
+
+
+INDEXER_DESCRIPTION = ("B=32, 8192-token contexts, top-512 of 64 heads x 128 bf16 dims, "
+                       "paged keys (4096 pages, 67 MB)")
+
+
+def make_indexer_config(seed: int | None = None) -> IndexerWorkload:
+    """The full-size indexer workload: batch 32 (the pages' steady batch),
+    contexts of 8,192 tokens (the pages' context cap), top-512."""
+    return indexer_workload(32, 8192, 4096, seed=1007 if seed is None else seed, topk=512, name="indexer")
 
 
 def indexer_algorithmic_bytes(w: IndexerWorkload) -> int:

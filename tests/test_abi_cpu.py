@@ -192,3 +192,44 @@ def test_decode_host_rejects_bad_arguments_before_any_copy():
     assert _host(s, st=None) == WORKSPACE
     assert _host(s, st=128) == WORKSPACE                 # staging not 256-byte aligned
     assert _host(s, nbytes=api.host_staging_size(s) - 1) == WORKSPACE
+
+
+# ------------------------------------------------------------ indexer
+def _ix_shape(**kw):
+    d = dict(batch=2, topk=16, max_ctx=256, pages_per_seq=4, num_key_rows=64 * 8)
+    d.update(kw)
+    s = api.indexer_shape(d.pop("batch"), d.pop("topk"), d.pop("max_ctx"), d.pop("pages_per_seq"),
+                          d.pop("num_key_rows"))
+    for k, v in d.items():
+        setattr(s, k, v)
+    return s
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(batch=0), INVALID), (dict(topk=0), INVALID), (dict(topk=65537), INVALID), (dict(max_ctx=0), INVALID),
+    (dict(max_ctx=(1 << 20) + 1), INVALID), (dict(reserved=1), INVALID), (dict(heads=32), UNSUPPORTED),
+    (dict(dim=64), UNSUPPORTED), (dict(page_size=32), UNSUPPORTED), (dict(pages_per_seq=3), INVALID),
+    (dict(num_key_rows=100), INVALID), (dict(num_key_rows=0), INVALID),
+])
+def test_indexer_bad_shapes_rejected_without_cuda(kw, code):
+    s = _ix_shape(**kw)
+    assert api.lib.sparse_mla_indexer_scores(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None) == code
+    assert api.lib.sparse_mla_indexer_topk(ctypes.byref(s), 16, 16, 16, None) == code
+    assert api.lib.sparse_mla_indexer(ctypes.byref(s), 16, 16, 16, 16, 16, 16, 16, None) == code
+
+
+def test_indexer_null_and_misaligned_pointers_rejected():
+    s = _ix_shape()
+    f = api.lib.sparse_mla_indexer_scores
+    assert f(None, 16, 16, 16, 16, 16, 16, None) == INVALID
+    for i in range(6):
+        args = [16] * 6
+        args[i] = None
+        assert f(ctypes.byref(s), *args, None) == INVALID
+    assert f(ctypes.byref(s), 8, 16, 16, 16, 16, 16, None) == INVALID     # q not 16-byte aligned
+    assert f(ctypes.byref(s), 16, 16, 8, 16, 16, 16, None) == INVALID     # keys not 16-byte aligned
+    assert f(ctypes.byref(s), 16, 2, 16, 16, 16, 16, None) == INVALID     # w not 4-byte aligned
+    g = api.lib.sparse_mla_indexer_topk
+    assert g(ctypes.byref(s), None, 16, 16, None) == INVALID
+    assert g(ctypes.byref(s), 16, 16, 2, None) == INVALID
+    assert api.lib.sparse_mla_indexer(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, None) == INVALID
