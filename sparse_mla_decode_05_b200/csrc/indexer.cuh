@@ -208,20 +208,86 @@ __device__ __forceinline__ int block_prefix_count(bool flag, int* sums, int* tot
   return r;
 }
 
+// Warp 0 (t < 32) of a top-k CTA: given the histogram of one 8-bit digit
+// over the keys still in play, the digit that holds the need-th largest key
+// (*s_digit) and how many keys equal to the selection are still to take
+// among those with that digit (*s_need).  Lane l holds digits 255 - 8 l ..
+// 248 - 8 l, highest first.
+__device__ __forceinline__ void radix_pick(const uint32_t* hist, int need, uint32_t* s_digit, int* s_need) {
+  const int t = threadIdx.x;
+  uint32_t c[8], sum = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    c[k] = hist[255 - 8 * t - k];
+    sum += c[k];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (t >= o) incl += v;
+  }
+  const uint32_t before = incl - sum;   // keys in higher digits
+  if (before < (uint32_t)need && (uint32_t)need <= incl) {
+    uint32_t acc = before;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (acc + c[k] >= (uint32_t)need) {
+        *s_digit = 255u - 8u * (uint32_t)t - (uint32_t)k;
+        *s_need = need - (int)acc;
+        break;
+      }
+      acc += c[k];
+    }
+  }
+}
+
+// Warp 0: exclusive prefix sums, in place, of the 256 counts v[0 .. 255];
+// returns the total to every lane of warp 0.
+__device__ __forceinline__ int prefix256(int* v) {
+  const int lane = threadIdx.x & 31;
+  int x[8], sum = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    x[k] = v[8 * lane + k];
+    sum += x[k];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    v[8 * lane + k] = run;
+    run += x[k];
+  }
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
 // One CTA per sequence.  Radix select of the topk-th largest key, 8 bits per
 // pass from the top (histograms in shared memory, one atomic per run of
 // equal digits in a warp); then the positions above that key, and the
 // lowest positions equal to it until topk are taken, written in ascending
-// order through block-wide prefix counts.
+// order.  Contexts up to 8,192 keep their keys in registers (position
+// k * 1024 + thread, k < 8): one read of the scores, and the ordered
+// compaction ranks by (k, warp, lane) through two 256-entry prefix sums.
+// Longer contexts re-read the scores each pass and compact 1,024 positions
+// at a time.
+constexpr int kTkPer = 8;   // keys per thread in registers
+
 __global__ void __launch_bounds__(kTkThreads) smla_topk_kernel(const float* __restrict__ scores,
                                                                const int32_t* __restrict__ ctx_len, int max_ctx,
                                                                int topk, int32_t* __restrict__ out) {
   __shared__ uint32_t hist[256];
+  __shared__ int cnt[256];            // [k][warp] counts, then their prefix sums
   __shared__ int sums[65];
   __shared__ uint32_t s_digit;
   __shared__ int s_need;
   grid_dep_wait();   // the scores come from the previous kernel
-  const int b = blockIdx.x, t = threadIdx.x, lane = t & 31;
+  const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   int n = __ldg(ctx_len + b);
   if (n < 0 || n > max_ctx) {
     if (t == 0) atomicOr(&g_error_word, 4u);
@@ -235,10 +301,75 @@ __global__ void __launch_bounds__(kTkThreads) smla_topk_kernel(const float* __re
   }
   uint32_t prefix = 0, mask = 0;
   int need = topk;   // keys still to take among those matching prefix
+  const uint32_t lt = (1u << lane) - 1u;
+  if (n <= kTkThreads * kTkPer) {
+    uint32_t key[kTkPer];
+#pragma unroll
+    for (int k = 0; k < kTkPer; ++k) {
+      const int i = k * kTkThreads + t;
+      key[k] = i < n ? order_key(row[i]) : 0u;
+    }
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      if (t < 256) hist[t] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < kTkPer; ++k) {
+        const bool in = k * kTkThreads + t < n && (key[k] & mask) == prefix;
+        const uint32_t digit = (key[k] >> shift) & 255u;
+        const unsigned act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const unsigned same = __match_any_sync(act, digit);
+          if (lane == __ffs(same) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(same));
+        }
+      }
+      __syncthreads();
+      if (t < 32) radix_pick(hist, need, &s_digit, &s_need);
+      __syncthreads();
+      prefix |= s_digit << shift;
+      mask |= 255u << shift;
+      need = s_need;
+      __syncthreads();
+    }
+    // ties: rank of each key equal to the selection among them, by position
+    unsigned eqm[kTkPer], selm[kTkPer];
+#pragma unroll
+    for (int k = 0; k < kTkPer; ++k) {
+      eqm[k] = __ballot_sync(0xffffffffu, k * kTkThreads + t < n && key[k] == prefix);
+      if (lane == 0) cnt[k * 32 + warp] = __popc(eqm[k]);
+    }
+    __syncthreads();
+    if (t < 32) prefix256(cnt);
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kTkPer; ++k) {
+      const bool valid = k * kTkThreads + t < n;
+      const bool eq = (eqm[k] >> lane) & 1u;
+      const int eq_rank = cnt[k * 32 + warp] + __popc(eqm[k] & lt);
+      selm[k] = __ballot_sync(0xffffffffu, valid && (key[k] > prefix || (eq && eq_rank < need)));
+    }
+    __syncthreads();   // every eq rank read before cnt is reused
+#pragma unroll
+    for (int k = 0; k < kTkPer; ++k)
+      if (lane == 0) cnt[k * 32 + warp] = __popc(selm[k]);
+    __syncthreads();
+    if (t < 32) prefix256(cnt);
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kTkPer; ++k) {
+      if ((selm[k] >> lane) & 1u) {
+        const int pos = cnt[k * 32 + warp] + __popc(selm[k] & lt);
+        if (pos < topk) orow[pos] = k * kTkThreads + t;
+      }
+    }
+    if (t == 0) grid_dep_launch();
+    return;
+  }
 #pragma unroll 1
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = t; i < 256; i += kTkThreads) hist[i] = 0;
+    if (t < 256) hist[t] = 0;
     __syncthreads();
 #pragma unroll 1
     for (int base = 0; base < n; base += kTkThreads) {
@@ -253,34 +384,7 @@ __global__ void __launch_bounds__(kTkThreads) smla_topk_kernel(const float* __re
       }
     }
     __syncthreads();
-    if (t < 32) {
-      // lane l holds digits 255 - 8 l .. 248 - 8 l (highest first)
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        c[k] = hist[255 - 8 * t - k];
-        sum += c[k];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (t >= o) incl += v;
-      }
-      const uint32_t before = incl - sum;   // keys in higher digits
-      if (before < (uint32_t)need && (uint32_t)need <= incl) {
-        uint32_t acc = before;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (acc + c[k] >= (uint32_t)need) {
-            s_digit = 255u - 8u * (uint32_t)t - (uint32_t)k;
-            s_need = need - (int)acc;
-            break;
-          }
-          acc += c[k];
-        }
-      }
-    }
+    if (t < 32) radix_pick(hist, need, &s_digit, &s_need);
     __syncthreads();
     prefix |= s_digit << shift;
     mask |= 255u << shift;
