@@ -242,6 +242,51 @@ __device__ __forceinline__ void radix_pick(const uint32_t* hist, int need, uint3
   }
 }
 
+// The same over 2,048 bins (an 11-bit digit), by all 1,024 threads of the
+// block: thread t holds bins 2047 - 2 t and 2046 - 2 t (highest first); a
+// warp scan and a scan of the 32 warp totals give each thread the number of
+// keys in higher bins.  Also sets *s_cnt, the keys that carry the chosen
+// digit.  wsum: 32 ints of shared memory.  Ends with the block synchronised.
+__device__ __forceinline__ void radix_pick2048(const uint32_t* hist, int need, int* wsum, uint32_t* s_digit,
+                                               int* s_need, int* s_cnt) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int c0 = (int)hist[2047 - 2 * t], c1 = (int)hist[2046 - 2 * t];
+  const int sum = c0 + c1;
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = wsum[lane];
+    int wi = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    __syncwarp();
+    wsum[lane] = wi - v;   // keys in the bins of lower-numbered warps
+  }
+  __syncthreads();
+  const int before = wsum[warp] + incl - sum;
+  if (before < need && need <= before + sum) {
+    if (before + c0 >= need) {
+      *s_digit = 2047u - 2u * (uint32_t)t;
+      *s_need = need - before;
+      *s_cnt = c0;
+    } else {
+      *s_digit = 2046u - 2u * (uint32_t)t;
+      *s_need = need - before - c0;
+      *s_cnt = c1;
+    }
+  }
+  __syncthreads();
+}
+
 // Warp 0: exclusive prefix sums, in place, of the 256 counts v[0 .. 255];
 // returns the total to every lane of warp 0.
 __device__ __forceinline__ int prefix256(int* v) {
@@ -267,27 +312,29 @@ __device__ __forceinline__ int prefix256(int* v) {
   return __shfl_sync(0xffffffffu, incl, 31);
 }
 
-// One CTA per sequence.  Radix select of the topk-th largest key, 8 bits per
-// pass from the top (histograms in shared memory, one atomic per run of
-// equal digits in a warp); then the positions above that key, and the
-// lowest positions equal to it until topk are taken, written in ascending
-// order.  Contexts up to 8,192 keep their keys in registers (position
-// k * 1024 + thread, k < 8): one read of the scores, and the ordered
-// compaction ranks by (k, warp, lane) through two 256-entry prefix sums.
-// Longer contexts re-read the scores each pass and compact 1,024 positions
-// at a time.
+// One CTA per sequence.  Radix select of the topk-th largest key, digit by
+// digit from the top (histograms in shared memory); then the positions
+// above that key, and the lowest positions equal to it until topk are
+// taken, written in ascending order.  Contexts up to 8,192 keep their keys
+// in registers (position k * 1024 + thread, k < 8): one read of the scores,
+// three digits of 11/11/10 bits, and an ordered compaction that ranks by
+// (k, warp, lane) through 256-entry prefix sums of per-warp ballot counts.
+// Longer contexts re-read the scores for each of four 8-bit digits (one
+// atomic per run of equal digits in a warp) and compact 1,024 positions at
+// a time.
 constexpr int kTkPer = 8;   // keys per thread in registers
 
-__global__ void __launch_bounds__(kTkThreads) smla_topk_kernel(const float* __restrict__ scores,
+__global__ void __launch_bounds__(kTkThreads, 1) smla_topk_kernel(const float* __restrict__ scores,
                                                                const int32_t* __restrict__ ctx_len, int max_ctx,
                                                                int topk, int32_t* __restrict__ out) {
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[2048];
   __shared__ int cnt[256];            // [k][warp] counts, then their prefix sums
   __shared__ int sums[65];
   __shared__ uint32_t s_digit;
-  __shared__ int s_need;
+  __shared__ int s_need, s_cnt;
   grid_dep_wait();   // the scores come from the previous kernel
   const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (t == 0) SMLA_TRACE_EV(0);
   int n = __ldg(ctx_len + b);
   if (n < 0 || n > max_ctx) {
     if (t == 0) atomicOr(&g_error_word, 4u);
@@ -309,47 +356,60 @@ __global__ void __launch_bounds__(kTkThreads) smla_topk_kernel(const float* __re
       const int i = k * kTkThreads + t;
       key[k] = i < n ? order_key(row[i]) : 0u;
     }
+    if (t == 0) SMLA_TRACE_EV(1 + (key[0] & 0u));
+    // three digits of 11, 11 and 10 bits: the top digit spans the sign,
+    // the exponent and two mantissa bits, so keys of one magnitude still
+    // spread over several bins (fewer colliding atomics than 8-bit digits)
+    int eq_count = 0;
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      if (t < 256) hist[t] = 0;
+    for (int pass = 0; pass < 3; ++pass) {
+      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+      const uint32_t dmask = pass == 2 ? 1023u : 2047u;
+      hist[t] = 0;
+      hist[t + 1024] = 0;
       __syncthreads();
+      // one shared-memory atomic per key: with 11-bit digits the keys of a
+      // warp spread over many bins, so same-address conflicts stay few
 #pragma unroll
       for (int k = 0; k < kTkPer; ++k) {
         const bool in = k * kTkThreads + t < n && (key[k] & mask) == prefix;
-        const uint32_t digit = (key[k] >> shift) & 255u;
-        const unsigned act = __ballot_sync(0xffffffffu, in);
-        if (in) {
-          const unsigned same = __match_any_sync(act, digit);
-          if (lane == __ffs(same) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(same));
-        }
+        if (in) atomicAdd(&hist[(key[k] >> shift) & dmask], 1u);
       }
       __syncthreads();
-      if (t < 32) radix_pick(hist, need, &s_digit, &s_need);
-      __syncthreads();
+      radix_pick2048(hist, need, sums, &s_digit, &s_need, &s_cnt);
       prefix |= s_digit << shift;
-      mask |= 255u << shift;
+      mask |= dmask << shift;
       need = s_need;
+      eq_count = s_cnt;
       __syncthreads();
+      if (t == 0) SMLA_TRACE_EV(2 + pass);
     }
-    // ties: rank of each key equal to the selection among them, by position
-    unsigned eqm[kTkPer], selm[kTkPer];
+    unsigned selm[kTkPer];
+    if (eq_count == need) {
+      // every key equal to the selection is taken (the usual case)
 #pragma unroll
-    for (int k = 0; k < kTkPer; ++k) {
-      eqm[k] = __ballot_sync(0xffffffffu, k * kTkThreads + t < n && key[k] == prefix);
-      if (lane == 0) cnt[k * 32 + warp] = __popc(eqm[k]);
-    }
-    __syncthreads();
-    if (t < 32) prefix256(cnt);
-    __syncthreads();
+      for (int k = 0; k < kTkPer; ++k)
+        selm[k] = __ballot_sync(0xffffffffu, k * kTkThreads + t < n && key[k] >= prefix);
+    } else {
+      // ties: rank of each key equal to the selection among them, by position
+      unsigned eqm[kTkPer];
 #pragma unroll
-    for (int k = 0; k < kTkPer; ++k) {
-      const bool valid = k * kTkThreads + t < n;
-      const bool eq = (eqm[k] >> lane) & 1u;
-      const int eq_rank = cnt[k * 32 + warp] + __popc(eqm[k] & lt);
-      selm[k] = __ballot_sync(0xffffffffu, valid && (key[k] > prefix || (eq && eq_rank < need)));
+      for (int k = 0; k < kTkPer; ++k) {
+        eqm[k] = __ballot_sync(0xffffffffu, k * kTkThreads + t < n && key[k] == prefix);
+        if (lane == 0) cnt[k * 32 + warp] = __popc(eqm[k]);
+      }
+      __syncthreads();
+      if (t < 32) prefix256(cnt);
+      __syncthreads();
+#pragma unroll
+      for (int k = 0; k < kTkPer; ++k) {
+        const bool valid = k * kTkThreads + t < n;
+        const bool eq = (eqm[k] >> lane) & 1u;
+        const int eq_rank = cnt[k * 32 + warp] + __popc(eqm[k] & lt);
+        selm[k] = __ballot_sync(0xffffffffu, valid && (key[k] > prefix || (eq && eq_rank < need)));
+      }
+      __syncthreads();   // every eq rank read before cnt is reused
     }
-    __syncthreads();   // every eq rank read before cnt is reused
 #pragma unroll
     for (int k = 0; k < kTkPer; ++k)
       if (lane == 0) cnt[k * 32 + warp] = __popc(selm[k]);
@@ -363,6 +423,7 @@ __global__ void __launch_bounds__(kTkThreads) smla_topk_kernel(const float* __re
         if (pos < topk) orow[pos] = k * kTkThreads + t;
       }
     }
+    if (t == 0) SMLA_TRACE_EV(6);
     if (t == 0) grid_dep_launch();
     return;
   }
