@@ -95,6 +95,7 @@ def _check(w, plan):
     (1, 128, 1, None, 4),        # one tile, top-1
     (2, 8192, 512, 4000, 300),   # long contexts, several thousand candidates
     (5, 2048, 2048, 1500, 200),  # top-k equal to the score row
+    (2, 12000, 512, 9000, 400),  # contexts past 8192: the top-k path that re-reads the scores
 ])
 def test_indexer_parity(B, max_ctx, topk, ctx_lo, pages):
     w = inputs.indexer_workload(B, max_ctx, pages, seed=B * 1000 + topk, topk=topk, ctx_lo=ctx_lo)
@@ -141,6 +142,20 @@ def test_ties_go_to_the_lower_position():
     got, sel = _check(w, plan)
     assert sel[1].tolist() == list(range(500))
     assert len(np.unique(got[0, :4096])) <= 5
+
+
+def test_ties_past_8192_positions():
+    """The long-context top-k path with the boundary inside a tie."""
+    w = inputs.indexer_workload(1, 10000, 160, seed=93, topk=700)
+    rows0 = ix.key_rows(w.page_table[0].numpy(), 10000)
+    pick = np.random.default_rng(93).integers(0, 7, size=10000)
+    k = w.k.clone()
+    k[torch.from_numpy(rows0)] = k[torch.from_numpy(rows0[:7][pick])]
+    w.k = k
+    plan = _plan(w)
+    plan.run()
+    got, _ = _check(w, plan)
+    assert len(np.unique(got[0, :10000])) <= 7
 
 
 def test_context_longer_than_the_row_is_clamped():
