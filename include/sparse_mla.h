@@ -41,8 +41,11 @@
  *  - Arguments are validated on the host before any launch.  On a
  *    validation error nothing is launched and no CUDA call is made.
  *  - Index values outside [-1, num_kv_rows) (flat) or
- *    [-1, pages_per_seq * page_size) (paged), and page-table entries outside
- *    the pool, are caller errors that the kernels do not check.
+ *    [-1, pages_per_seq * page_size) (paged), and page-table entries that
+ *    point outside the pool, are caller errors.  The kernels check every
+ *    entry as they resolve it: such an entry is read as padding (it takes no
+ *    part and nothing is read for it) and sets bit 2 of the device error
+ *    word (sparse_mla_get_device_error).
  *  - Entry points are thread-safe; they keep no per-call state.
  */
 #ifndef SPARSE_MLA_H_
@@ -92,7 +95,7 @@ typedef enum {
 typedef struct {
   int32_t batch;          /* B >= 1: sequences, one query token each          */
   int32_t num_heads;      /* H = 64                                            */
-  int32_t d_qk;           /* 576 = 512 latent + 64 rope                        */
+  int32_t d_qk;           /* 576 = 512 latent + 64 rope (512 for DSV4 pages)   */
   int32_t d_v;            /* 512: the value is the first 512 dims of the row   */
   int32_t topk;           /* k >= 1 entries in each index list                 */
   int32_t kv_dtype;       /* smla_kv_dtype                                     */
@@ -198,10 +201,16 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
 
 /* Reads and clears the library's device error word on the current device
  * (a synchronous device-to-host copy: call it outside timed or captured
- * regions).  *code receives the raw word (0 = no error; bit 0: a kernel gave
- * up waiting on a pipeline barrier; bit 1: misaligned shared memory window;
- * bit 2: an index entry named no row of the pool and was read as padding).  Returns SMLA_ERR_DEVICE_TIMEOUT if
- * the word was non-zero, SMLA_OK if zero, SMLA_ERR_CUDA on a copy failure. */
+ * regions).  *code receives the raw word, 0 = no error:
+ *   bit 0  a kernel gave up a bounded wait on a pipeline barrier
+ *   bit 1  the shared-memory window was not 1024-byte aligned (the kernel
+ *          returned without computing)
+ *   bit 2  an input named something outside its range and was read as
+ *          absent: a decode index entry or page-table entry outside the
+ *          pool, an indexer context length outside [0, max_ctx] (clamped)
+ *          or an indexer page-table entry outside the key cache.
+ * Returns SMLA_ERR_DEVICE_TIMEOUT if the word was non-zero, SMLA_OK if zero,
+ * SMLA_ERR_CUDA on a copy failure. */
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
 /* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:
