@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) smla_topk_kernel(const float* _
       const int i = k * kTkThreads + t;
       key[k] = i < n ? order_key(row[i]) : 0u;
     }
-    if (t == 0) SMLA_TRACE_EV(1 + (key[0] & 0u));
+    if (t == 0) SMLA_TRACE_EV(1);
     // three digits of 11, 11 and 10 bits: the top digit spans the sign,
     // the exponent and two mantissa bits, so keys of one magnitude still
     // spread over several bins (fewer colliding atomics than 8-bit digits)
