@@ -32,7 +32,9 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for must in ("sparse_mla_decode", "sparse_mla_decode_split", "sparse_mla_combine",
                  "sparse_mla_workspace_size", "sparse_mla_plan_nsplit", "sparse_mla_status_string",
-                 "sparse_mla_abi_version", "sparse_mla_get_device_error"):
+                 "sparse_mla_abi_version", "sparse_mla_get_device_error", "sparse_mla_plan_merge",
+                 "sparse_mla_decode_static_scratch", "sparse_mla_decode_host", "sparse_mla_host_staging_size",
+                 "sparse_mla_indexer", "sparse_mla_indexer_scores", "sparse_mla_indexer_topk"):
         assert must in names
 
 
@@ -52,6 +54,9 @@ def test_abi_version_and_status_strings():
 def test_struct_layout_matches_header():
     assert ctypes.sizeof(api.SmlaShape) == 48
     assert api.SmlaShape.num_kv_rows.offset == 24
+    # smla_indexer_shape: eight int32 fields, then the int64 row count
+    assert ctypes.sizeof(api.IndexerShape) == 40
+    assert api.IndexerShape.num_key_rows.offset == 32
 
 
 def _decode(shape, q=16, kv=16, rs=None, pt=None, idx=16, scale=0.04, out=16, lse=16, ws=None, nbytes=0):
