@@ -41,6 +41,10 @@ static_assert(kIxSmemK % 1024 == 0 && kIxAtomQ % 1024 == 0 && kIxAtomK % 1024 ==
 
 constexpr int kTkThreads = 1024;                 // top-k: one CTA per sequence
 
+// the C ABI struct as the Python binding lays it out
+static_assert(sizeof(smla_indexer_shape) == 40 && offsetof(smla_indexer_shape, num_key_rows) == 32,
+              "smla_indexer_shape layout");
+
 struct IndexerParams {
   const uint8_t* q;            // [B, 64, 128] bf16
   const float* w;              // [B, 64]
