@@ -19,7 +19,9 @@ Keys beyond the base contract:
                copied host -> device from pinned memory and out / lse back
                inside the timed region of every step; the value pipelines
                steps over four streams (serial: one stream, in "serial")
-  per_config   microseconds per call and GB/s for every workload, vs roofline
+  per_config   microseconds per call and GB/s for every workload (the six
+               headline configs, DeepSeek-V4 pages, and the indexer step
+               that produces the index lists), vs roofline
   clocks       SM clock / throttle reasons sampled during the timed region
 """
 from __future__ import annotations
