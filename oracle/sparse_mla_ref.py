@@ -54,6 +54,7 @@ __all__ = [
     "gather_rows_f64",
     "attend_rows",
     "sparse_mla_decode",
+    "sparse_mla_decode_multi_token",
     "combine_partials",
 ]
 
@@ -271,6 +272,28 @@ def sparse_mla_decode(q_bits: np.ndarray, kv: np.ndarray, indices: np.ndarray,
         k = gather_rows_f64(kv, rows, kv_format=kv_format, row_scale=kv_row_scale)
         qh = bf16_bits_to_f64(q_bits[b])
         out[b], lse[b] = attend_rows(qh, k, scale, d_v)
+    return out, lse
+
+
+def sparse_mla_decode_multi_token(q_bits: np.ndarray, kv: np.ndarray, indices: np.ndarray, scale: float, *,
+                                  d_v: int = 512, kv_format: str = "bf16", kv_row_scale: np.ndarray | None = None,
+                                  page_table: np.ndarray | None = None, page_size: int = 0):
+    """fp64 decode of s_q query tokens per sequence (speculative / multi-token
+    decode): token t of sequence b attends over its own index list
+    indices[b, t] through the sequence's page table, exactly as one decode
+    token does.  A list shared by all tokens is the special case.
+
+    q_bits  [B, s_q, H, d_qk] uint16, indices [B, s_q, k] int32,
+    page_table [B, pages_per_seq] int32 when page_size > 0.
+    Returns out [B, s_q, H, d_v] and lse [B, s_q, H] (float64)."""
+    q_bits = np.asarray(q_bits)
+    B, T, H, d_qk = q_bits.shape
+    out = np.empty((B, T, H, d_v))
+    lse = np.empty((B, T, H))
+    for t in range(T):
+        out[:, t], lse[:, t] = sparse_mla_decode(q_bits[:, t], kv, np.asarray(indices)[:, t], scale, d_v=d_v,
+                                                 kv_format=kv_format, kv_row_scale=kv_row_scale,
+                                                 page_table=page_table, page_size=page_size)
     return out, lse
 
 
