@@ -58,7 +58,7 @@
 extern "C" {
 #endif
 
-#define SMLA_ABI_VERSION 1
+#define SMLA_ABI_VERSION 2
 
 typedef enum {
   SMLA_OK = 0,
@@ -66,8 +66,13 @@ typedef enum {
   SMLA_ERR_UNSUPPORTED = 2,    /* shape this build does not implement        */
   SMLA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than required */
   SMLA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed       */
-  SMLA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait (see
+  SMLA_ERR_DEVICE_TIMEOUT = 5, /* a kernel gave up a bounded wait (see
                                   sparse_mla_get_device_error)              */
+  SMLA_ERR_DEVICE_INDEX = 6,   /* a kernel met an index, page-table entry or
+                                  context length outside its range and read
+                                  it as absent (error word bit 2 alone)     */
+  SMLA_ERR_DEVICE_LAYOUT = 7   /* a kernel found its shared-memory window
+                                  misaligned and computed nothing (bit 1)   */
 } smla_status;
 
 typedef enum {
@@ -209,8 +214,9 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
  *          absent: a decode index entry or page-table entry outside the
  *          pool, an indexer context length outside [0, max_ctx] (clamped)
  *          or an indexer page-table entry outside the key cache.
- * Returns SMLA_ERR_DEVICE_TIMEOUT if the word was non-zero, SMLA_OK if zero,
- * SMLA_ERR_CUDA on a copy failure. */
+ * Returns, for the most serious bit set: SMLA_ERR_DEVICE_TIMEOUT (bit 0),
+ * SMLA_ERR_DEVICE_LAYOUT (bit 1), SMLA_ERR_DEVICE_INDEX (bit 2); SMLA_OK if
+ * the word was zero; SMLA_ERR_CUDA on a copy failure. */
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
 /* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:

@@ -20,7 +20,8 @@ KV_BF16, KV_FP8_E4M3_ROWSCALE, KV_DSV4_PAGED = 0, 1, 2
 DSV4_PAGE_BYTES, DSV4_D_QK = 37376, 512   # DeepSeek-V4 page: 64 x 576 slot bytes + 64 x 8 scale bytes
 
 STATUS = {0: "SMLA_OK", 1: "SMLA_ERR_INVALID_ARG", 2: "SMLA_ERR_UNSUPPORTED", 3: "SMLA_ERR_WORKSPACE",
-          4: "SMLA_ERR_CUDA", 5: "SMLA_ERR_DEVICE_TIMEOUT"}
+          4: "SMLA_ERR_CUDA", 5: "SMLA_ERR_DEVICE_TIMEOUT", 6: "SMLA_ERR_DEVICE_INDEX",
+          7: "SMLA_ERR_DEVICE_LAYOUT"}
 
 
 class SmlaError(RuntimeError):
@@ -261,7 +262,7 @@ def device_error() -> int:
     """Reads and clears the device error word (synchronous)."""
     code = ctypes.c_uint32(0)
     st = lib.sparse_mla_get_device_error(ctypes.byref(code))
-    if st not in (0, 5):
+    if st not in (0, 5, 6, 7):
         raise SmlaError(st, "sparse_mla_get_device_error")
     return code.value
 

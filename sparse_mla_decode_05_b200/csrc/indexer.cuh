@@ -338,7 +338,6 @@ __global__ void __launch_bounds__(kTkThreads, 1) smla_topk_kernel(const float* _
   __shared__ int s_need, s_cnt;
   grid_dep_wait();   // the scores come from the previous kernel
   const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  if (t == 0) SMLA_TRACE_EV(0);
   int n = __ldg(ctx_len + b);
   if (n < 0 || n > max_ctx) {
     if (t == 0) atomicOr(&g_error_word, 4u);
@@ -360,7 +359,6 @@ __global__ void __launch_bounds__(kTkThreads, 1) smla_topk_kernel(const float* _
       const int i = k * kTkThreads + t;
       key[k] = i < n ? order_key(row[i]) : 0u;
     }
-    if (t == 0) SMLA_TRACE_EV(1);
     // three digits of 11, 11 and 10 bits: the top digit spans the sign,
     // the exponent and two mantissa bits, so keys of one magnitude still
     // spread over several bins (fewer colliding atomics than 8-bit digits)
@@ -386,7 +384,6 @@ __global__ void __launch_bounds__(kTkThreads, 1) smla_topk_kernel(const float* _
       need = s_need;
       eq_count = s_cnt;
       __syncthreads();
-      if (t == 0) SMLA_TRACE_EV(2 + pass);
     }
     unsigned selm[kTkPer];
     if (eq_count == need) {
@@ -427,7 +424,6 @@ __global__ void __launch_bounds__(kTkThreads, 1) smla_topk_kernel(const float* _
         if (pos < topk) orow[pos] = k * kTkThreads + t;
       }
     }
-    if (t == 0) SMLA_TRACE_EV(6);
     if (t == 0) grid_dep_launch();
     return;
   }

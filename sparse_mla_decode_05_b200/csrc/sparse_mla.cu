@@ -15,16 +15,17 @@
 //    one program per head re-reading the same rows 64 times ([Diag] "The
 //    Subject Message"; [Design] "Design Decisions" 1).  Here one CTA owns
 //    (sequence, top-k chunk); 64-token tiles are gathered into shared memory
-//    with 16-byte cp.async (fp8 rows: register loads + exact fp8->bf16
-//    conversion) and consumed by the tensor cores for every head.
+//    with 16-byte cp.async (fp8 rows: codes copied, then converted exactly
+//    to bf16 in shared memory) and consumed by the tensor cores for every
+//    head.
 //  * Scores and PV as tensor-core contractions across the head group with
 //    fp32 accumulation ([Design] "Design Decisions" 5-6).  Here: tcgen05.mma
 //    with accumulators in tensor memory (TMEM):
-//        S  = Q . K^T     M = 64 heads, N = 64 tokens, K = 576   (TMEM, fp32)
-//        O^T += V^T . P^T M = 128 dims (x4 chunks), N = 64 heads, K = 64 tokens
-//    The whole 64x576 query lives in shared memory next to two tile buffers:
-//    B200's 227 KB per CTA lets BLOCK_H = 64 (all heads) fit, which the
-//    pages' ~99 KB sm_120 budget forbade ([Design] "Memory Budgeting").
+//        S  = Q . K^T   M = 64 heads, N = 64 tokens, K = 576, Q read from TMEM
+//        O += P . V     M = 64 heads, N = 2 x 256 dims, K = 64 tokens
+//    The query sits in tensor memory and three 64-row tiles in shared
+//    memory: B200's 227 KB per CTA lets BLOCK_H = 64 (all heads) fit, which
+//    the pages' ~99 KB sm_120 budget forbade ([Design] "Memory Budgeting").
 //  * Online softmax in fp32; masked entries (index -1) take no part
 //    ([Design] "Edge Case Handling").  Rows of masked entries are zero-filled
 //    in shared memory and their probabilities are exactly 0.
@@ -36,8 +37,10 @@
 //
 // Warp roles in the split kernel (one CTA per SM; ~227 KB shared memory):
 //   warps 0-3  softmax + epilogue (128 threads; warp w owns TMEM lanes 32w..)
-//   warp  4    TMEM allocator; lane 0 issues every tcgen05.mma
-//   warps 5..  producers: resolve indices (flat or paged), gather rows
+//   warp  4    TMEM allocator; issues S = Q K^T
+//   warp  5    issues O += P V
+//   warps 6-9  resolve indices (flat or paged) to rows
+//   warps 10.. gather rows (and, for fp8 codes, convert them)
 // Every wait on a pipeline barrier is bounded (about 2 s): on expiry the CTA
 // records an error bit in a device word, drains its own copies and MMAs,
 // frees TMEM and exits.
@@ -66,43 +69,42 @@ constexpr int kTileBytes = kAtoms * kAtomBytes;     // 73,728
 constexpr int kRowBytesBf16 = kDqk * 2;             // 1152
 constexpr int kRowBytesFp8 = kDqk;                  // 576
 
-// shared memory map (offsets from the 1024-aligned dynamic shared base)
-constexpr int kStages = 3;                          // KV tile stages
-constexpr int kSmemKV = 0;                          // KV  [3 stages][9 atoms][64 tok][128 B]
-// P(t) [64 heads][64 tok] bf16 (K-major) takes the place of the rope atom of
-// the stage that holds tile t: S(t) has read that atom by the time P(t) is
-// written, PV(t) reads the rest of the stage, and the stage is refilled only
-// after PV(t).  Each stage thus carries its own P buffer.
+constexpr int kRawRowBytes = 576;                   // fp8 row / DeepSeek-V4 slot (codes as stored)
+constexpr int kRawTileBytes = kTile * kRawRowBytes; // 36,864
+
+// Shared memory map (offsets from the 1024-aligned dynamic shared base):
+//   [operand stages][raw stages][aux]
+// Operand stage: one 64-row tile as bf16, 9 atoms of [64 rows][128 B],
+// 128-byte swizzled (K-major for S, MN-major for PV).  P(t) [64 heads][64
+// tok] bf16 (K-major) takes the place of the rope atom of the stage that
+// holds tile t: S(t) has read that atom by the time P(t) is written, PV(t)
+// reads the rest of the stage, and the stage is refilled only after PV(t).
+// Each stage thus carries its own P buffer.
+// Raw stage (fp8 / DeepSeek-V4 caches): one tile's rows as stored, 576
+// contiguous bytes per row, before conversion to bf16.
+constexpr int kSmemKV = 0;
 constexpr int kAtomP = kAtoms - 1;
-constexpr int kSmemAux = kSmemKV + kStages * kTileBytes;
 constexpr int kRing = 4;                            // resolved-row ring depth (tiles)
+constexpr int kMaxStages = 3;
 // barrier indices
-constexpr int BAR_KVF = 0;                          // [kStages] tile landed
-constexpr int BAR_KVE = BAR_KVF + kStages;          // [kStages] tile consumed (PV done)
-constexpr int BAR_SF = BAR_KVE + kStages;           // [2] S(t) in TMEM
+constexpr int BAR_KVF = 0;                          // [stages] operand tile ready
+constexpr int BAR_KVE = BAR_KVF + kMaxStages;       // [stages] operand tile consumed (PV done)
+constexpr int BAR_SF = BAR_KVE + kMaxStages;        // [2] S(t) in TMEM
 constexpr int BAR_SE = BAR_SF + 2;                  // [2] S(t) read by the softmax
-constexpr int BAR_PF = BAR_SE + 2;                  // [kStages] P(t) written (per stage)
-constexpr int BAR_PVD = BAR_PF + kStages;           // [2] PV(t) done (by tile parity)
+constexpr int BAR_PF = BAR_SE + 2;                  // [stages] P(t) written (per stage)
+constexpr int BAR_PVD = BAR_PF + kMaxStages;        // [2] PV(t) done (by tile parity)
 constexpr int BAR_FIN = BAR_PVD + 2;                // drain, S issuer
 constexpr int BAR_FIN2 = BAR_FIN + 1;               // drain, PV issuer
 constexpr int BAR_QT = BAR_FIN2 + 1;                // query written to TMEM
 constexpr int BAR_QS = BAR_QT + 1;                  // query staged in shared memory
 constexpr int BAR_PVI = BAR_QS + 1;                 // [2] PV(t) issued (by tile parity)
 constexpr int BAR_IXF = BAR_PVI + 2;                // [kRing] rows resolved
-constexpr int BAR_IXS = BAR_IXF + kRing;            // [kRing] fp8 row scales resolved
+constexpr int BAR_IXS = BAR_IXF + kRing;            // [kRing] row scales / scale blocks resolved
 constexpr int BAR_IXE = BAR_IXS + kRing;            // [kRing] rows consumed
-constexpr int BAR_RAW = BAR_IXE + kRing;            // [kStages] fp8 codes landed
-constexpr int BAR_CS1 = BAR_RAW + kStages;          // cluster: every split's blocks written
+constexpr int BAR_RAW = BAR_IXE + kRing;            // [raw stages] raw rows landed
+constexpr int BAR_RAWE = BAR_RAW + kMaxStages;      // [raw stages] raw rows converted
+constexpr int BAR_CS1 = BAR_RAWE + kMaxStages;      // cluster: every split's blocks written
 constexpr int kNumBars = BAR_CS1 + 1;
-constexpr int kAuxBars = kSmemAux;
-constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
-constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
-constexpr int kAuxRsc = kAuxRow + kRing * 64 * 4;   // f32  [kRing][64] fp8 row scales
-constexpr int kAuxDsc = kAuxRsc + kRing * 64 * 4;   // u64  [kRing][64] DeepSeek-V4 scale blocks
-constexpr int kAuxEnd = kAuxDsc + kRing * 64 * 8;
-constexpr int kSmemBytes = kAuxEnd;
-static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
-static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxDsc % 16 == 0, "aux arrays are read as vectors");
 // DeepSeek-V4 page: 64 slots of 576 bytes (448 e4m3fn codes, 64 bf16), then
 // 64 scale blocks of 8 bytes (7 UE8M0 exponents, one per 64 code dims)
 constexpr int kDsv4Slot = 576, kDsv4Nope = 448;
@@ -137,10 +139,9 @@ constexpr uint32_t kIdescPV = make_idesc(64, 256, false, true);   // O += P V   
 constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // warps 0-3 softmax/epilogue, 4 S-MMA issuer (+ TMEM allocator), 5 PV-MMA
-// issuer, 6-9 index resolvers (warp 6+k owns the tiles t = k mod 4), 10..
-// loaders: copy warps issuing 16-byte cp.async (bf16 rows: four warps; fp8
-// codes: two warps), then, for fp8 only, eight warps that convert the codes
-// to bf16 in place
+// issuer, 6-9 index resolvers (warp 6+k owns the tiles t = k mod 4), 10-13
+// copy warps, then, for fp8 and DeepSeek-V4 caches, four warps that convert
+// the raw codes to bf16 operand tiles
 constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kIdxWarps = 4, kWarpLoad0 = kWarpIdx + kIdxWarps;
 // the in-cluster merge uses warps 0-7 and, for the lse, index warps 8-9
 static_assert(kWarpIdx <= 8 && kWarpIdx + kIdxWarps >= 10, "warps 8 and 9 must be index warps");
@@ -150,12 +151,32 @@ constexpr int kKindFp8 = 1;    // e4m3fn rows [N, 576] + one fp32 scale per row
 constexpr int kKindDsv4 = 2;   // DeepSeek-V4 pages: 448 e4m3fn + UE8M0 group scales, 64 bf16 rope
 template <int kKind>
 struct Cfg {
-  static constexpr bool kConv = kKind != kKindBf16;     // codes converted to bf16 by convert warps
-  static constexpr int kCopyWarps = kConv ? 2 : 4;
-  static constexpr int kCvtWarps = kConv ? 8 : 0;
+  static constexpr bool kConv = kKind != kKindBf16;     // raw codes converted to bf16 by convert warps
+  static constexpr int kStages = kConv ? 2 : 3;         // operand stages
+  static constexpr int kRawStages = kConv ? 2 : 0;      // raw stages
+  static constexpr int kQStage = kStages - 1;           // holds the staged query until it is in TMEM
+  static constexpr int kCopyWarps = 4;
+  static constexpr int kCvtWarps = kConv ? 4 : 0;
   static constexpr int kCopyThreads = kCopyWarps * 32;
   static constexpr int kLoadWarps = kCopyWarps + kCvtWarps;
   static constexpr int kThreads = (kWarpLoad0 + kLoadWarps) * 32;
+  // Raw tiles: 8-row groups g < kCpGroups arrive by 16-byte cp.async, the
+  // rest by one bulk copy per row (the copy engine adds bandwidth to the
+  // load/store path's); copy warp w owns the groups g = w mod 4.
+  static constexpr int kCpGroups = kConv ? 5 : 8;
+  static constexpr int kBulkWarps = kConv ? (8 - kCpGroups < 4 ? 8 - kCpGroups : 4) : 0;
+  // shared memory map
+  static constexpr int kSmemRaw = kSmemKV + kStages * kTileBytes;
+  static constexpr int kSmemAux = kSmemRaw + kRawStages * kRawTileBytes;
+  static constexpr int kAuxBars = kSmemAux;
+  static constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
+  static constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
+  static constexpr int kAuxRsc = kAuxRow + kRing * 64 * 4;   // f32  [kRing][64] fp8 row scales
+  static constexpr int kAuxDsc = kAuxRsc + kRing * 64 * 4;   // u64  [kRing][64] DeepSeek-V4 scale blocks
+  static constexpr int kSmemBytes = kAuxDsc + kRing * 64 * 8;
+  static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
+  static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxDsc % 16 == 0, "aux arrays are read as vectors");
+  static_assert(kCopyWarps == 4 && kCpGroups >= 4 && kCpGroups <= 8, "copy-warp group ownership");
 };
 
 struct SplitParams {
@@ -184,11 +205,6 @@ static __device__ __align__(256) unsigned char g_static_scratch[SMLA_STATIC_SCRA
 // ---------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -482,18 +498,6 @@ __device__ __forceinline__ uint32_t sw128_off(int r, int j) {
 }
 
 // ============================================================ split kernel
-#ifdef SMLA_TRACE
-// Development-only timeline probe (compiled only with -DSMLA_TRACE): the
-// global timer at fixed pipeline events of the first 256 CTAs.
-__device__ unsigned long long g_trace[256 * 64];
-#define SMLA_TRACE_EV(ev)                                                          \
-  do {                                                                             \
-    const int cta_ = blockIdx.y * gridDim.x + blockIdx.x;                          \
-    if (cta_ < 256 && (ev) < 64) g_trace[cta_ * 64 + (ev)] = globaltimer_ns();     \
-  } while (0)
-#else
-#define SMLA_TRACE_EV(ev) do { } while (0)
-#endif
 
 __device__ __forceinline__ void bulk_store_s2g(void* gdst, uint32_t ssrc, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
@@ -634,14 +638,16 @@ __device__ __forceinline__ void merge_tail(const float* wss, const uint4* wso, i
 template <int kKind>
 __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     smla_split_kernel(const __grid_constant__ SplitParams p) {
-  constexpr int kCopy = Cfg<kKind>::kCopyThreads;
+  using C = Cfg<kKind>;
+  constexpr int kCopy = C::kCopyThreads;
   constexpr bool kFp8 = kKind == kKindFp8;     // row scale folded into S and P
   constexpr bool kDsv4 = kKind == kKindDsv4;
-  constexpr bool kConv = Cfg<kKind>::kConv;
+  constexpr bool kConv = C::kConv;
+  constexpr int kStages = C::kStages;
   constexpr int kQK = kDsv4 ? 512 : kDqk;      // query / key width
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bars = sbase + kAuxBars;
+  const uint32_t bars = sbase + C::kAuxBars;
   auto BAR = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5;
@@ -660,22 +666,26 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     if (threadIdx.x == 0) atomicOr(&g_error_word, 2u);
     return;
   }
-  SMLA_TRACE_EV(0);
 
-  int* s_row = reinterpret_cast<int*>(smem + kAuxRow);
-  float* s_rsc = reinterpret_cast<float*>(smem + kAuxRsc);
-  uint2* s_dsc = reinterpret_cast<uint2*>(smem + kAuxDsc);
+  int* s_row = reinterpret_cast<int*>(smem + C::kAuxRow);
+  float* s_rsc = reinterpret_cast<float*>(smem + C::kAuxRsc);
+  uint2* s_dsc = reinterpret_cast<uint2*>(smem + C::kAuxDsc);
 
   if (threadIdx.x == 0) {
     // Arrivals are per warp (the warp synchronises, one lane arrives), except
     // where a copy engine arrives: mbarrier arrivals are serialised.
     for (int s = 0; s < kStages; ++s) {
-      // bf16: one arrival per copying thread (when its copies land); fp8:
-      // one per convert warp
-      mbar_init(BAR(BAR_KVF + s), kConv ? Cfg<kKind>::kCvtWarps : kCopy);
-      mbar_init(BAR(BAR_RAW + s), kCopy);
+      // bf16: one arrival per copying thread (when its copies land); fp8 /
+      // DeepSeek-V4: one per convert warp
+      mbar_init(BAR(BAR_KVF + s), kConv ? C::kCvtWarps : kCopy);
       mbar_init(BAR(BAR_KVE + s), 1);
       mbar_init(BAR(BAR_PF + s), 4);
+    }
+    for (int s = 0; s < C::kRawStages; ++s) {
+      // one arrival per copying thread when its cp.async land, plus one
+      // expect-tx arrival per warp that issues bulk copies
+      mbar_init(BAR(BAR_RAW + s), kCopy + C::kBulkWarps);
+      mbar_init(BAR(BAR_RAWE + s), C::kCvtWarps);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(BAR_SF + s), 1);
@@ -692,14 +702,13 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       mbar_init(BAR(BAR_IXF + r), 1);
       mbar_init(BAR(BAR_IXS + r), 1);
       // consumers of a ring slot: the copy warps (rows), the softmax warps
-      // (row scales) and, for DeepSeek-V4 pages, the convert warps (scale
-      // blocks)
-      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + 4 + (kDsv4 ? Cfg<kKind>::kCvtWarps : 0));
+      // (row scales) and the convert warps (rows to zero, scale blocks)
+      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + 4 + C::kCvtWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == kWarpS) {
-    tmem_alloc(sbase + kAuxTmem, kTmemCols);
+    tmem_alloc(sbase + C::kAuxTmem, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -711,8 +720,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
   // dependent launch all of it overlapped the previous kernel
   grid_dep_wait();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kAuxTmem);
-  SMLA_TRACE_EV(1);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::kAuxTmem);
 
   bool merge_failed = false;   // a softmax warp gave up (in-cluster merge)
   if (warp >= kWarpIdx && warp < kWarpIdx + kIdxWarps) {
@@ -743,12 +751,12 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       return (int)r;
     };
     const int kw = warp - kWarpIdx;
-    // the 64 x kQK query (contiguous bf16) into the third KV stage, which
-    // no tile uses before the query has been moved to tensor memory
+    // the 64 x kQK query (contiguous bf16) into the last operand stage,
+    // which no tile uses before the query has been moved to tensor memory
     if (kw == 0 && lane == 0) {
       constexpr uint32_t kQBytes = (uint32_t)kH * kQK * 2;
       mbar_arrive_expect_tx(BAR(BAR_QS), kQBytes);
-      bulk_load_g2s(sbase + kSmemKV + 2 * kTileBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
+      bulk_load_g2s(sbase + kSmemKV + C::kQStage * kTileBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
     }
     // Software pipeline over this warp's tiles (step S = 4), every load
     // consumed one iteration after it was issued: index of tile t+3S, page
@@ -804,144 +812,170 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXS + rs));
-      if (lane == 0 && t < 4) SMLA_TRACE_EV(58 + t);
       r0_0 = r1_0; r0_1 = r1_1;
       c0_0 = c1_0; c0_1 = c1_1;
       d0_0 = d1_0; d0_1 = d1_1;
       r1_0 = r2_0; r1_1 = r2_1;
       i2_0 = i3_0; i2_1 = i3_1;
     }
-  } else if (warp >= kWarpLoad0 + Cfg<kKind>::kCopyWarps) {
-    // ------------------------------------------------- fp8 convert warps
-    // Thread (tok, sub) turns the 16 codes of dims [16 sub, 16 sub + 16) of
-    // every atom into bf16.  The copy warps put those codes in the first of
-    // the two 16-byte chunks their bf16 values occupy in the swizzled tile,
-    // so each thread reads and rewrites only its own two chunks: the
-    // conversion runs in place with no barrier between threads.
-    const int ct = threadIdx.x - 32 * (kWarpLoad0 + Cfg<kKind>::kCopyWarps);  // 0 .. 255
+  } else if (kConv && warp >= kWarpLoad0 + C::kCopyWarps) {
+    // ------------------------------------------------------- convert warps
+    // fp8 / DeepSeek-V4 caches: turn raw tile t (rows as stored, 576
+    // contiguous bytes each) into bf16 operand tile t.  Thread (tok, sub)
+    // converts the 16 codes of dims [64 a + 16 sub, +16) of every atom a of
+    // rows tok and tok + 32 (one 16-byte load, two 16-byte stores per atom;
+    // a warp's eight rows alternate between the two halves of a 128-byte
+    // bank window on the load side and spread over the swizzle on the store
+    // side).  Padding rows are written as zeros, whatever the raw slot holds.
+    const int ct = threadIdx.x - 32 * (kWarpLoad0 + C::kCopyWarps);  // 0 .. 127
+    const int tok0 = ct >> 2, sub = ct & 3;
     // DeepSeek-V4 pages: atoms 0..6 hold codes (times the group's UE8M0
     // scale), atom 7 the bf16 rope dims, copied as they are
-    const int tok = ct >> 2, sub = ct & 3;
     constexpr int kCvtAtoms = kDsv4 ? kDsv4Nope / 64 : kAtoms;
+    constexpr int kRaw = C::kRawStages > 0 ? C::kRawStages : 1;   // (compiled for every kind)
     for (int t = 0; t < ntiles; ++t) {
-      const int stage = t % kStages;
-      uint2 dsc = make_uint2(0u, 0u);
-      if constexpr (kDsv4) {
-        const int rs = t % kRing;
-        if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXS + rs), (t / kRing) & 1))) break;
-        dsc = s_dsc[rs * 64 + tok];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-      }
-      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + stage), (t / kStages) & 1))) break;
-      if (ct == 0 && t < 8) SMLA_TRACE_EV(40 + t);
+      const int stage = t % kStages, rst = t % kRaw, rs = t % kRing;
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXS + rs), (t / kRing) & 1))) break;
+      const bool valid0 = s_row[rs * 64 + tok0] >= 0, valid1 = s_row[rs * 64 + tok0 + 32] >= 0;
+      const uint2 dsc0 = kDsv4 ? s_dsc[rs * 64 + tok0] : make_uint2(0u, 0u);
+      const uint2 dsc1 = kDsv4 ? s_dsc[rs * 64 + tok0 + 32] : make_uint2(0u, 0u);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + rst), (t / kRaw) & 1))) break;
+      if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+        break;
+      // the last operand stage first holds the staged query
+      if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0))) break;
+      const uint32_t rbase = sbase + C::kSmemRaw + rst * kRawTileBytes;
       const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
-      const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
-      // all loads first (independent), then convert and store
-      uint4 v[kCvtAtoms];
+#pragma unroll 1
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int tok = tok0 + 32 * h2;
+        const bool valid = h2 ? valid1 : valid0;
+        const uint2 dsc = h2 ? dsc1 : dsc0;
+        const uint32_t src = rbase + tok * kRawRowBytes + sub * 16;
+        const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
+        // all loads first (independent), then convert and store
+        uint4 v[kCvtAtoms];
 #pragma unroll
-      for (int a = 0; a < kCvtAtoms; ++a) v[a] = ld_shared_v4(tbase + a * kAtomBytes + lo_off);
+        for (int a = 0; a < kCvtAtoms; ++a) v[a] = ld_shared_v4(src + a * 64);
 #pragma unroll
-      for (int a = 0; a < kCvtAtoms; ++a) {
-        uint4 lo, hi;
-        if constexpr (kDsv4) {
-          const uint32_t s2 = ue8m0_bf16x2(((a < 4 ? dsc.x : dsc.y) >> (8 * (a & 3))) & 0xFFu);
-          e4m3x4_to_bf16x4_scaled(v[a].x, s2, lo.x, lo.y);
-          e4m3x4_to_bf16x4_scaled(v[a].y, s2, lo.z, lo.w);
-          e4m3x4_to_bf16x4_scaled(v[a].z, s2, hi.x, hi.y);
-          e4m3x4_to_bf16x4_scaled(v[a].w, s2, hi.z, hi.w);
-        } else {
-          e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
-          e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
-          e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
-          e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
+        for (int a = 0; a < kCvtAtoms; ++a) {
+          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = make_uint4(0u, 0u, 0u, 0u);
+          if (valid) {
+            if constexpr (kDsv4) {
+              const uint32_t s2 = ue8m0_bf16x2(((a < 4 ? dsc.x : dsc.y) >> (8 * (a & 3))) & 0xFFu);
+              e4m3x4_to_bf16x4_scaled(v[a].x, s2, lo.x, lo.y);
+              e4m3x4_to_bf16x4_scaled(v[a].y, s2, lo.z, lo.w);
+              e4m3x4_to_bf16x4_scaled(v[a].z, s2, hi.x, hi.y);
+              e4m3x4_to_bf16x4_scaled(v[a].w, s2, hi.z, hi.w);
+            } else {
+              e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
+              e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
+              e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
+              e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
+            }
+          }
+          st_shared_v4(tbase + a * kAtomBytes + lo_off, lo);
+          st_shared_v4(tbase + a * kAtomBytes + hi_off, hi);
         }
-        st_shared_v4(tbase + a * kAtomBytes + lo_off, lo);
-        st_shared_v4(tbase + a * kAtomBytes + hi_off, hi);
+        if constexpr (kDsv4) {
+          // rope: bf16 bytes [448 + 32 sub, +32) of the slot, chunks 2 sub
+          // and 2 sub + 1 of atom 7
+          uint4 lo = ld_shared_v4(rbase + tok * kRawRowBytes + kDsv4Nope + 32 * sub);
+          uint4 hi = ld_shared_v4(rbase + tok * kRawRowBytes + kDsv4Nope + 32 * sub + 16);
+          if (!valid) lo = hi = make_uint4(0u, 0u, 0u, 0u);
+          st_shared_v4(tbase + 7 * kAtomBytes + lo_off, lo);
+          st_shared_v4(tbase + 7 * kAtomBytes + hi_off, hi);
+        }
       }
       // one proxy fence for the tile: generic stores -> tensor-core reads
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(BAR_KVF + stage));
-      if (ct == 0 && (t == 2 || t == 3)) SMLA_TRACE_EV(t == 2 ? 57 : 63);
+      if (lane == 0) {
+        mbar_arrive(BAR(BAR_KVF + stage));
+        mbar_arrive(BAR(BAR_RAWE + rst));
+      }
     }
   } else if (warp >= kWarpLoad0) {
     // ------------------------------------------------------- copy warps
+    // Each warp instruction covers eight rows, four 16-byte chunks of each
+    // (lane = 4 row + chunk): spreading an instruction over many rows keeps
+    // more DRAM requests independent, which measured faster on B200 than
+    // whole-row instructions.  Copy warp lw owns the 8-row groups g = lw and
+    // lw + 4 of every tile.  Padding rows read nothing (source size 0).
     const int lt = threadIdx.x - 32 * kWarpLoad0;  // 0 .. kCopy-1
     const int lw = lt >> 5;
+    const int r8 = lane >> 2, c4 = lane & 3;
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages, rs = t % kRing;
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1))) break;  // warp-uniform
-      const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
-      // bf16: lane covers tokens 4u + lane/8, 16-byte chunk lane%8 of a
-      // 128-byte atom row; fp8: tokens 8(4 lw + u) + lane/4, 16 codes
-      // (chunk lane%4) of a 64-byte atom row
-      int rows[16];
-      if constexpr (!kConv) {
+      // this lane's row in groups lw and lw + 4, and, for a bulk group, the
+      // row of lane l < 8
+      int rows[2], brow[2];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) rows[u] = s_row[rs * 64 + 4 * u + (lane >> 3)];
-      } else {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) rows[u] = s_row[rs * 64 + 4 * (8 * lw + u) + (lane >> 3)];
+      for (int gi = 0; gi < 2; ++gi) {
+        rows[gi] = s_row[rs * 64 + 8 * (lw + 4 * gi) + r8];
+        brow[gi] = s_row[rs * 64 + 8 * (lw + 4 * gi) + (lane & 7)];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-      if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
-        break;
-      // stage 2 first holds the staged query
-      if (__any_sync(0xffffffffu, t == 2 && !mbar_wait(BAR(BAR_QT), 0))) break;
       if constexpr (!kConv) {
-        if (lt == 0 && t < 8) SMLA_TRACE_EV(40 + t);
-        // warp w copies atoms w, w+4, w+8; each warp instruction covers four
-        // whole 128-byte row segments (coalesced); padding rows are
-        // zero-filled (source size 0)
-        const int j = lane & 7;
-#pragma unroll 1
-        for (int a = lw; a < kAtoms; a += 4) {
+        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+          break;
+        // the last stage first holds the staged query
+        if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0))) break;
+        // bf16 rows straight into the swizzled operand tile: chunk c (0..71)
+        // of a row is 16-byte chunk c % 8 of atom c / 8
+        const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int tok = 4 * u + (lane >> 3);
-            const int row = rows[u];
-            const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16 + a * 128 + j * 16;
-            cp_async_16(tbase + a * kAtomBytes + sw128_off(tok, j), src, row >= 0 ? 16u : 0u);
+        for (int gi = 0; gi < 2; ++gi) {
+          const int tok = 8 * (lw + 4 * gi) + r8;
+          const int row = rows[gi];
+          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16;
+          const uint32_t nbytes = row >= 0 ? 16u : 0u;
+#pragma unroll
+          for (int sg = 0; sg < 18; ++sg) {
+            const int c = 4 * sg + c4;
+            cp_async_16(tbase + (c >> 3) * kAtomBytes + sw128_off(tok, c & 7), src + c * 16, nbytes);
           }
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
       } else {
-        if (lt == 0 && t < 8) SMLA_TRACE_EV(48 + t);
-        // each warp instruction covers four whole 128-byte row segments
-        // (a row is 4.5 segments); 16-code chunk c of a row goes to the first
-        // chunk of its bf16 destination (atom c / 4, see the convert warps).
-        // A DeepSeek-V4 slot is also 576 bytes: chunks 0..27 are codes, and
-        // the 64 bf16 rope dims (bytes 448..575) go straight to atom 7, lane
-        // j of a row's eight lanes copying rope chunk j.
-        const int j = lane & 7;
+        // raw rows, 576 contiguous bytes each, into raw stage t % 2: groups
+        // g < kCpGroups by cp.async, the others one bulk copy per row
+        const int rst = t % C::kRawStages;
+        if (__any_sync(0xffffffffu, t >= C::kRawStages &&
+                                        !mbar_wait(BAR(BAR_RAWE + rst), ((t / C::kRawStages) - 1) & 1)))
+          break;
+        const uint32_t rbase = sbase + C::kSmemRaw + rst * kRawTileBytes;
+        auto row_src = [&](int r) -> const uint8_t* {
+          if constexpr (kDsv4) return p.kv + (size_t)(r >> 6) * kDsv4Page + (r & 63) * kDsv4Slot;
+          else return p.kv + (size_t)r * kRowBytesFp8;
+        };
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int tok = 4 * (8 * lw + u) + (lane >> 3);
-          const int row = rows[u];
-          const int rr = row >= 0 ? row : 0;
-          const uint32_t nbytes = row >= 0 ? 16u : 0u;
-          if constexpr (kDsv4) {
-            const uint8_t* src = p.kv + (size_t)(rr >> 6) * kDsv4Page + (rr & 63) * kDsv4Slot;
-#pragma unroll
-            for (int sg = 0; sg < 4; ++sg) {
-              const int c = 8 * sg + j;
-              if (c < kDsv4Nope / 16)
-                cp_async_16(tbase + (c >> 2) * kAtomBytes + sw128_off(tok, 2 * (c & 3)), src + c * 16, nbytes);
-            }
-            cp_async_16(tbase + 7 * kAtomBytes + sw128_off(tok, j), src + kDsv4Nope + j * 16, nbytes);
+        for (int gi = 0; gi < 2; ++gi) {
+          const int g = lw + 4 * gi;
+          if (g >= C::kCpGroups) {
+            // bulk group: lane l < 8 copies row 8 g + l when it is valid
+            const bool v = lane < 8 && brow[gi] >= 0;
+            const uint32_t nv = __popc(__ballot_sync(0xffffffffu, v));
+            if (lane == 0) mbar_arrive_expect_tx(BAR(BAR_RAW + rst), nv * (uint32_t)kRawRowBytes);
+            __syncwarp();
+            if (v) bulk_load_g2s(rbase + (8 * g + lane) * kRawRowBytes, row_src(brow[gi]), kRawRowBytes, BAR(BAR_RAW + rst));
           } else {
-            const uint8_t* src = p.kv + (size_t)rr * kRowBytesFp8;
+            const int tok = 8 * g + r8;
+            const int row = rows[gi];
+            const uint8_t* src = row_src(row >= 0 ? row : 0);
+            const uint32_t nbytes = row >= 0 ? 16u : 0u;
 #pragma unroll
-            for (int sg = 0; sg < 5; ++sg) {
-              const int c = 8 * sg + j;
-              if (c < kRowBytesFp8 / 16)
-                cp_async_16(tbase + (c >> 2) * kAtomBytes + sw128_off(tok, 2 * (c & 3)), src + c * 16, nbytes);
+            for (int sg = 0; sg < 9; ++sg) {
+              const int c = 4 * sg + c4;
+              cp_async_16(rbase + tok * kRawRowBytes + c * 16, src + c * 16, nbytes);
             }
           }
         }
-        cp_async_mbar_arrive_noinc(BAR(BAR_RAW + stage));
+        cp_async_mbar_arrive_noinc(BAR(BAR_RAW + rst));
       }
     }
     cp_async_wait_all();
@@ -958,12 +992,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     };
     bool ok = true;
     if (warp == kWarpS) {
-      uint64_t dk[kStages];
-#pragma unroll
-      for (int s = 0; s < kStages; ++s) dk[s] = sw128_desc(sbase + kSmemKV + s * kTileBytes, 16, 1024);
+      const uint64_t dk0 = sw128_desc(sbase + kSmemKV, 16, 1024);
       ok = wait_all(BAR(BAR_QT), 0);
       tc_fence_after();
-      if (lane == 0) SMLA_TRACE_EV(2);
       for (int t = 0; ok && t < ntiles; ++t) {
         const int stage = t % kStages, sb = t & 1;
         // S(t) reuses the S buffer of S(t-2): its softmax must have read it.
@@ -977,8 +1008,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         }
         ok = wait_all(BAR(BAR_KVF + stage), (t / kStages) & 1);
         if (!ok) break;
-        if (lane == 0 && t < 8) SMLA_TRACE_EV(24 + t);
-        const uint64_t bk = stage == 0 ? dk[0] : (stage == 1 ? dk[1] : dk[2]);
+        // stage s starts s * kTileBytes later (descriptor address field: bytes >> 4)
+        const uint64_t bk = dk0 + (uint64_t)(stage * (kTileBytes >> 4));
         const uint32_t d = tmem + kColS + 64u * (uint32_t)sb;
         // 36 K steps: Q columns +8 per step (16 bf16); K descriptor: atom
         // +512, 16-element step +2
@@ -989,19 +1020,16 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
           mma_ts_acc_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + off, kIdescS);
         }
         commit_elect(BAR(BAR_SF + sb));
-        if (lane == 0 && t < 8) SMLA_TRACE_EV(8 + t);
       }
     } else {
-      uint64_t dv[kStages];
-#pragma unroll
-      for (int s = 0; s < kStages; ++s) dv[s] = sw128_desc(sbase + kSmemKV + s * kTileBytes, kAtomBytes, 1024);
+      const uint64_t dv0 = sw128_desc(sbase + kSmemKV, kAtomBytes, 1024);
       const uint32_t o0 = tmem + (kLaneO << 16);
       for (int t = 0; ok && t < ntiles; ++t) {
         const int stage = t % kStages;
         ok = wait_all(BAR(BAR_PF + stage), (t / kStages) & 1);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t bv = stage == 0 ? dv[0] : (stage == 1 ? dv[1] : dv[2]);
+        const uint64_t bv = dv0 + (uint64_t)(stage * (kTileBytes >> 4));
         // P(t) sits in the stage's rope atom
         const uint64_t dp = sw128_desc(sbase + kSmemKV + stage * kTileBytes + kAtomP * kAtomBytes, 16, 1024);
         // O[:, 256 hf + n] += P[:, 16 kk + k] V[16 kk + k, 256 hf + n]:
@@ -1022,7 +1050,6 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         commit_elect(BAR(BAR_PVD + (t & 1)));
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(BAR_PVI + (t & 1)));
-        if (lane == 0 && t < 8) SMLA_TRACE_EV(16 + t);
       }
     }
     // drain: every MMA this warp issued has completed before teardown
@@ -1040,7 +1067,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
        // from the copy staged in shared memory (row-major [64][kQK])
       bool okq = mbar_wait(BAR(BAR_QS), 0);
       if (okq) {
-        const uint8_t* qrow = smem + kSmemKV + 2 * kTileBytes + h * (kQK * 2) + half * kQK;
+        const uint8_t* qrow = smem + kSmemKV + C::kQStage * kTileBytes + h * (kQK * 2) + half * kQK;
 #pragma unroll 1
         for (int c = 0; c < kQK / 64; ++c) {
           uint32_t r[16];
@@ -1154,7 +1181,6 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_PF + i % kStages));
-      if (threadIdx.x == 0 && i < 8) SMLA_TRACE_EV(32 + i);
     }
     // ---------------------------------------------------------- epilogue
     // this CTA's tiles are done: the next kernel of the stream may start
@@ -1167,7 +1193,6 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       aborted = __any_sync(0xffffffffu, aborted);
       tc_fence_after();
     }
-    if (threadIdx.x == 0) SMLA_TRACE_EV(3);
     if (p.cluster) {
       // in-cluster merge (after the warp roles): this split's per-head
       // statistics (max, fp32 sum, rounded-P sum) go to the workspace
@@ -1178,7 +1203,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
         *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4) = make_float4(m_run, l_nrm, l_tot, 0.f);
         // for the merge writers: 1 / (rounded-P sum) of head h
-        reinterpret_cast<float*>(smem + kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
+        reinterpret_cast<float*>(smem + C::kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
       }
     } else if (!aborted) {
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
@@ -1234,7 +1259,6 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         else p.part_lse[part * kH + h] = lse_h;
         bulk_wait_all();
       }
-      if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     }
     tc_fence_before();
   }
@@ -1271,15 +1295,13 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // every PV has completed (the PV issuer's drain barrier: one phase)
       failed = !mbar_wait(BAR(BAR_FIN2), 0);
       tc_fence_after();
-      if (lane == 0 && warp == 4) SMLA_TRACE_EV(52);
     }
     const bool bad = group_any(failed, 1, 256);
-    if (threadIdx.x == 0) SMLA_TRACE_EV(48);
     if (!bad) {
       // this split's result for the thread's head, normalised by its own
       // rounded-P sum (a convex combination of value rows) and rounded to
       // fp16: 11 significant bits, error <= 2^-12 of the largest value
-      const float sc = reinterpret_cast<const float*>(smem + kAuxRow)[16 * q + (lane & 15)];
+      const float sc = reinterpret_cast<const float*>(smem + C::kAuxRow)[16 * q + (lane & 15)];
       uint4* mine = wso + (size_t)split * kSplitU + (size_t)q * (8 * 4 * 32) + lane;
       const uint32_t olanes = (uint32_t)(32 * q + kLaneO) << 16;
       float o[2][32];
@@ -1304,21 +1326,16 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         if (ntiles > 0 && cc + 1 < 4) tmem_wait_ld();
       }
     }
-    if (threadIdx.x == 0) SMLA_TRACE_EV(49);
     named_bar_sync(1, 256);
-    if (threadIdx.x == 0) SMLA_TRACE_EV(50);
     // lane r of warp 0 arrives on CTA r's barrier: the n remote arrivals go
     // out together (one after another they cost a round trip each)
     // (each arrival is a cluster-scope release: after the CTA barrier it
     // covers every merging thread's stores)
     if (warp == 0) {
-      if (lane == 0) SMLA_TRACE_EV(51);
       if (lane < n) mbar_arrive_cluster(mapa_shared(BAR(BAR_CS1), (uint32_t)lane));
       __syncwarp();
     }
-    if (threadIdx.x == 0) SMLA_TRACE_EV(4);
     const bool ok = mbar_wait_cluster(BAR(BAR_CS1), 0);
-    if (threadIdx.x == 0) SMLA_TRACE_EV(7);
     if (!group_any(bad || !ok, 1, 256)) {
       const int hh = 16 * q + (lane & 15);
       const int part = (lane >> 4) + 2 * upper;
@@ -1331,9 +1348,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         case 8: merge_tail<8>(wss, wso, q, lane, hh, col0, orow); break;
         default: merge_tail<16>(wss, wso, q, lane, hh, col0, orow); break;
       }
-      if (threadIdx.x == 0) SMLA_TRACE_EV(62);
     }
-    if (threadIdx.x == 0) SMLA_TRACE_EV(5);
     tc_fence_before();
   } else if (p.cluster && split == 0 && warp >= 8 && warp < 10) {
     // lse of the merged result, head 32 (warp - 8) + lane, from every
@@ -1368,7 +1383,6 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  SMLA_TRACE_EV(6);
 }
 
 // ============================================================ combine kernel
@@ -1515,7 +1529,7 @@ static cudaError_t ensure_smem_attr() {
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
   const cudaError_t e =
-      cudaFuncSetAttribute(smla_split_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      cudaFuncSetAttribute(smla_split_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<kKind>::kSmemBytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
   return e;
 }
@@ -1547,7 +1561,7 @@ static const ClusterCaps& cluster_caps() {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(1u << lg, 1, 1);
       cfg.blockDim = dim3(Cfg<kKind>::kThreads, 1, 1);
-      cfg.dynamicSmemBytes = kSmemBytes;
+      cfg.dynamicSmemBytes = Cfg<kKind>::kSmemBytes;
       cfg.attrs = at;
       cfg.numAttrs = 1;
       int k = 0;
@@ -1587,7 +1601,7 @@ static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(prm.nsplit, prm.batch);
   cfg.blockDim = dim3(Cfg<kKind>::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = Cfg<kKind>::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = at;
   cfg.numAttrs = na;
@@ -1727,6 +1741,8 @@ const char* sparse_mla_status_string(smla_status s) {
     case SMLA_ERR_WORKSPACE: return "SMLA_ERR_WORKSPACE";
     case SMLA_ERR_CUDA: return "SMLA_ERR_CUDA";
     case SMLA_ERR_DEVICE_TIMEOUT: return "SMLA_ERR_DEVICE_TIMEOUT";
+    case SMLA_ERR_DEVICE_INDEX: return "SMLA_ERR_DEVICE_INDEX";
+    case SMLA_ERR_DEVICE_LAYOUT: return "SMLA_ERR_DEVICE_LAYOUT";
   }
   return "SMLA_ERR_UNKNOWN";
 }
@@ -1863,20 +1879,10 @@ smla_status sparse_mla_get_device_error(uint32_t* code) {
   const unsigned int zero = 0;
   if (w != 0 && cudaMemcpyToSymbol(smla::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SMLA_ERR_CUDA;
   if (code) *code = w;
-  return w ? SMLA_ERR_DEVICE_TIMEOUT : SMLA_OK;
+  if (w & 1u) return SMLA_ERR_DEVICE_TIMEOUT;
+  if (w & 2u) return SMLA_ERR_DEVICE_LAYOUT;
+  if (w & 4u) return SMLA_ERR_DEVICE_INDEX;
+  return SMLA_OK;
 }
 
 }  // extern "C"
-
-#ifdef SMLA_TRACE
-// Development-only accessor of the timeline probe (not part of the ABI).
-extern "C" int smla_trace_read(unsigned long long* host, size_t n) {
-  if (n > sizeof(smla::g_trace) / sizeof(unsigned long long)) n = sizeof(smla::g_trace) / sizeof(unsigned long long);
-  if (cudaMemcpyFromSymbol(host, smla::g_trace, n * sizeof(unsigned long long)) != cudaSuccess) return -1;
-  return (int)n;
-}
-extern "C" int smla_trace_clear(void) {
-  static unsigned long long zeros[256 * 64];
-  return cudaMemcpyToSymbol(smla::g_trace, zeros, sizeof(zeros)) == cudaSuccess ? 0 : -1;
-}
-#endif

@@ -350,6 +350,47 @@ def make_config(name: str, seed: int | None = None) -> Workload:
     raise KeyError(name)
 
 
+def reindexed(w: Workload, seed: int) -> Workload:
+    """Another batch of the same workload over the same cache: fresh queries
+    and fresh index lists drawn by ``w``'s own recipe (the pool, row scales
+    and page tables are shared, not copied).  Used to rotate distinct
+    batches through a timed loop so that successive steps gather different
+    rows of a pool larger than L2."""
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    m = w.meta
+    B, topk = w.batch, w.topk
+    q_mult = m.get("q_mult", 1.0)
+    q = _normal_bf16(gen, tuple(w.q.shape), mult=q_mult)
+    idx = np.full((B, topk), -1, dtype=np.int64)
+    if "lens" in m:                                   # flat_varlen
+        lens = np.asarray(m["lens"])
+        offs = np.concatenate([[0], np.cumsum(lens)[:-1]])
+        for b in range(B):
+            if lens[b] >= topk:
+                idx[b] = _distinct(rng, int(lens[b]), topk) + offs[b]
+            else:
+                idx[b, :lens[b]] = rng.permutation(int(lens[b])) + offs[b]
+    elif w.page_size:                                 # paged pools: logical positions
+        for b in range(B):
+            idx[b] = _distinct(rng, m["rows_per_seq"], topk)
+    else:                                             # flat_per_seq
+        R = m["rows_per_seq"]
+        for b in range(B):
+            if m.get("index_mode", "uniform") == "recency":
+                win = min(1024, R)
+                n_recent = topk // 2
+                recent = R - win + _distinct(rng, win, n_recent)
+                rest_pool = np.setdiff1d(np.arange(R), recent, assume_unique=True)
+                rest = rest_pool[_distinct(rng, rest_pool.size, topk - n_recent)]
+                sel = np.sort(np.concatenate([recent, rest]))
+            else:
+                sel = _distinct(rng, R, topk)
+            idx[b] = sel + b * R
+    return dataclasses.replace(w, q=q, indices=torch.from_numpy(idx.astype(np.int32)),
+                               meta=dict(m, reindexed_seed=seed))
+
+
 def shard_seed(name: str, rank: int) -> int | None:
     """Seed of rank ``rank``'s batch of workload ``name`` when the step runs
     as independent per-GPU batches (the op shards over sequences): rank 0

@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert api.lib.sparse_mla_abi_version() == 1
+    assert api.lib.sparse_mla_abi_version() == 2
     for code, name in api.STATUS.items():
         assert api.lib.sparse_mla_status_string(code).decode() == name
     assert api.lib.sparse_mla_status_string(99).decode() == "SMLA_ERR_UNKNOWN"

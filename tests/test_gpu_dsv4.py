@@ -166,6 +166,28 @@ def test_dsv4_single_index_is_the_decoded_row():
     assert ref.lse_rel_err(lse.cpu().numpy().astype(np.float64), lse_ref).max() <= 1e-3
 
 
+@pytest.mark.parametrize("nsplit", [0, 1, 4])
+def test_dsv4_rope_alone_decides(nsplit):
+    """Every nope code is zero, so the scores come from the 64 bf16 rope dims
+    alone and the output is zero except in dims 448..511, where it is a
+    softmax-weighted mean of rope values.  A rope chunk that is not copied,
+    or copied to the wrong place, changes both (checked against the oracle
+    at the usual bar), and the nope part of the output must be exactly 0."""
+    w = inputs.paged_dsv4(3, 2048, 96, 700, seed=77 + nsplit)
+    pages = w.kv.numpy().copy()
+    for sl in range(64):
+        pages[:, sl * SLOT:sl * SLOT + 448] = 0
+    w = inputs.Workload(name="dsv4_rope_only", q=w.q, kv=torch.from_numpy(pages), indices=w.indices,
+                        scale=w.scale, page_table=w.page_table, page_size=64, layout="dsv4")
+    d = Dev(w)
+    out, lse = d.run(nsplit=nsplit)
+    torch.cuda.synchronize()
+    out_ref, lse_ref = oracle(w)
+    assert np.abs(out_ref[..., 448:]).max() > 0.1          # the rope part carries the result
+    assert_parity(out, lse, out_ref, lse_ref, tag=f"dsv4 rope only n={nsplit}")
+    assert np.array_equal(out[..., :448].float().cpu().numpy(), np.zeros((3, 64, 448), dtype=np.float32))
+
+
 def test_dsv4_input_checks():
     w = inputs.paged_dsv4(2, 256, 16, 50, seed=3)
     d = Dev(w)
