@@ -155,16 +155,16 @@ struct Cfg {
   static constexpr int kStages = kConv ? 2 : 3;         // operand stages
   static constexpr int kRawStages = kConv ? 2 : 0;      // raw stages
   static constexpr int kQStage = kStages - 1;           // holds the staged query until it is in TMEM
-  static constexpr int kCopyWarps = 4;
-  static constexpr int kCvtWarps = kConv ? 4 : 0;
+  static constexpr int kCopyWarps = kConv ? 2 : 4;
+  static constexpr int kCvtWarps = kConv ? 8 : 0;
   static constexpr int kCopyThreads = kCopyWarps * 32;
   static constexpr int kLoadWarps = kCopyWarps + kCvtWarps;
   static constexpr int kThreads = (kWarpLoad0 + kLoadWarps) * 32;
   // Raw tiles: 8-row groups g < kCpGroups arrive by 16-byte cp.async, the
   // rest by one bulk copy per row (the copy engine adds bandwidth to the
-  // load/store path's); copy warp w owns the groups g = w mod 4.
+  // load/store path's); copy warp w owns the groups g = w mod kCopyWarps.
   static constexpr int kCpGroups = kConv ? 5 : 8;
-  static constexpr int kBulkWarps = kConv ? (8 - kCpGroups < 4 ? 8 - kCpGroups : 4) : 0;
+  static constexpr int kBulkGroups = 8 - kCpGroups;      // one expect-tx arrival each
   // shared memory map
   static constexpr int kSmemRaw = kSmemKV + kStages * kTileBytes;
   static constexpr int kSmemAux = kSmemRaw + kRawStages * kRawTileBytes;
@@ -176,7 +176,8 @@ struct Cfg {
   static constexpr int kSmemBytes = kAuxDsc + kRing * 64 * 8;
   static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
   static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxDsc % 16 == 0, "aux arrays are read as vectors");
-  static_assert(kCopyWarps == 4 && kCpGroups >= 4 && kCpGroups <= 8, "copy-warp group ownership");
+  static_assert(8 % kCopyWarps == 0 && kCpGroups >= 1 && kCpGroups <= 8, "copy-warp group ownership");
+  static_assert(!kConv || kCvtWarps == 8, "convert warps: one thread per (row, 16-code column)");
 };
 
 struct SplitParams {
@@ -683,8 +684,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     }
     for (int s = 0; s < C::kRawStages; ++s) {
       // one arrival per copying thread when its cp.async land, plus one
-      // expect-tx arrival per warp that issues bulk copies
-      mbar_init(BAR(BAR_RAW + s), kCopy + C::kBulkWarps);
+      // expect-tx arrival per 8-row group copied in bulk
+      mbar_init(BAR(BAR_RAW + s), kCopy + C::kBulkGroups);
       mbar_init(BAR(BAR_RAWE + s), C::kCvtWarps);
     }
     for (int s = 0; s < 2; ++s) {
@@ -823,22 +824,22 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // fp8 / DeepSeek-V4 caches: turn raw tile t (rows as stored, 576
     // contiguous bytes each) into bf16 operand tile t.  Thread (tok, sub)
     // converts the 16 codes of dims [64 a + 16 sub, +16) of every atom a of
-    // rows tok and tok + 32 (one 16-byte load, two 16-byte stores per atom;
-    // a warp's eight rows alternate between the two halves of a 128-byte
-    // bank window on the load side and spread over the swizzle on the store
-    // side).  Padding rows are written as zeros, whatever the raw slot holds.
-    const int ct = threadIdx.x - 32 * (kWarpLoad0 + C::kCopyWarps);  // 0 .. 127
-    const int tok0 = ct >> 2, sub = ct & 3;
+    // row tok (one 16-byte load, two 16-byte stores per atom; a warp's eight
+    // rows alternate between the two halves of a 128-byte bank window on the
+    // load side and spread over the swizzle on the store side).  Padding
+    // rows are written as zeros, whatever the raw slot holds.
+    const int ct = threadIdx.x - 32 * (kWarpLoad0 + C::kCopyWarps);  // 0 .. 255
+    const int tok = ct >> 2, sub = ct & 3;
     // DeepSeek-V4 pages: atoms 0..6 hold codes (times the group's UE8M0
     // scale), atom 7 the bf16 rope dims, copied as they are
     constexpr int kCvtAtoms = kDsv4 ? kDsv4Nope / 64 : kAtoms;
     constexpr int kRaw = C::kRawStages > 0 ? C::kRawStages : 1;   // (compiled for every kind)
+    const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages, rst = t % kRaw, rs = t % kRing;
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXS + rs), (t / kRing) & 1))) break;
-      const bool valid0 = s_row[rs * 64 + tok0] >= 0, valid1 = s_row[rs * 64 + tok0 + 32] >= 0;
-      const uint2 dsc0 = kDsv4 ? s_dsc[rs * 64 + tok0] : make_uint2(0u, 0u);
-      const uint2 dsc1 = kDsv4 ? s_dsc[rs * 64 + tok0 + 32] : make_uint2(0u, 0u);
+      const bool valid = s_row[rs * 64 + tok] >= 0;
+      const uint2 dsc = kDsv4 ? s_dsc[rs * 64 + tok] : make_uint2(0u, 0u);
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + rst), (t / kRaw) & 1))) break;
@@ -846,48 +847,40 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         break;
       // the last operand stage first holds the staged query
       if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0))) break;
-      const uint32_t rbase = sbase + C::kSmemRaw + rst * kRawTileBytes;
+      const uint32_t rrow = sbase + C::kSmemRaw + rst * kRawTileBytes + tok * kRawRowBytes;
       const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
-#pragma unroll 1
-      for (int h2 = 0; h2 < 2; ++h2) {
-        const int tok = tok0 + 32 * h2;
-        const bool valid = h2 ? valid1 : valid0;
-        const uint2 dsc = h2 ? dsc1 : dsc0;
-        const uint32_t src = rbase + tok * kRawRowBytes + sub * 16;
-        const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
-        // all loads first (independent), then convert and store
-        uint4 v[kCvtAtoms];
+      // all loads first (independent), then convert and store
+      uint4 v[kCvtAtoms];
 #pragma unroll
-        for (int a = 0; a < kCvtAtoms; ++a) v[a] = ld_shared_v4(src + a * 64);
+      for (int a = 0; a < kCvtAtoms; ++a) v[a] = ld_shared_v4(rrow + sub * 16 + a * 64);
 #pragma unroll
-        for (int a = 0; a < kCvtAtoms; ++a) {
-          uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = make_uint4(0u, 0u, 0u, 0u);
-          if (valid) {
-            if constexpr (kDsv4) {
-              const uint32_t s2 = ue8m0_bf16x2(((a < 4 ? dsc.x : dsc.y) >> (8 * (a & 3))) & 0xFFu);
-              e4m3x4_to_bf16x4_scaled(v[a].x, s2, lo.x, lo.y);
-              e4m3x4_to_bf16x4_scaled(v[a].y, s2, lo.z, lo.w);
-              e4m3x4_to_bf16x4_scaled(v[a].z, s2, hi.x, hi.y);
-              e4m3x4_to_bf16x4_scaled(v[a].w, s2, hi.z, hi.w);
-            } else {
-              e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
-              e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
-              e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
-              e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
-            }
+      for (int a = 0; a < kCvtAtoms; ++a) {
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) {
+          if constexpr (kDsv4) {
+            const uint32_t s2 = ue8m0_bf16x2(((a < 4 ? dsc.x : dsc.y) >> (8 * (a & 3))) & 0xFFu);
+            e4m3x4_to_bf16x4_scaled(v[a].x, s2, lo.x, lo.y);
+            e4m3x4_to_bf16x4_scaled(v[a].y, s2, lo.z, lo.w);
+            e4m3x4_to_bf16x4_scaled(v[a].z, s2, hi.x, hi.y);
+            e4m3x4_to_bf16x4_scaled(v[a].w, s2, hi.z, hi.w);
+          } else {
+            e4m3x4_to_bf16x4(v[a].x, lo.x, lo.y);
+            e4m3x4_to_bf16x4(v[a].y, lo.z, lo.w);
+            e4m3x4_to_bf16x4(v[a].z, hi.x, hi.y);
+            e4m3x4_to_bf16x4(v[a].w, hi.z, hi.w);
           }
-          st_shared_v4(tbase + a * kAtomBytes + lo_off, lo);
-          st_shared_v4(tbase + a * kAtomBytes + hi_off, hi);
         }
-        if constexpr (kDsv4) {
-          // rope: bf16 bytes [448 + 32 sub, +32) of the slot, chunks 2 sub
-          // and 2 sub + 1 of atom 7
-          uint4 lo = ld_shared_v4(rbase + tok * kRawRowBytes + kDsv4Nope + 32 * sub);
-          uint4 hi = ld_shared_v4(rbase + tok * kRawRowBytes + kDsv4Nope + 32 * sub + 16);
-          if (!valid) lo = hi = make_uint4(0u, 0u, 0u, 0u);
-          st_shared_v4(tbase + 7 * kAtomBytes + lo_off, lo);
-          st_shared_v4(tbase + 7 * kAtomBytes + hi_off, hi);
-        }
+        st_shared_v4(tbase + a * kAtomBytes + lo_off, lo);
+        st_shared_v4(tbase + a * kAtomBytes + hi_off, hi);
+      }
+      if constexpr (kDsv4) {
+        // rope: bf16 bytes [448 + 32 sub, +32) of the slot, chunks 2 sub and
+        // 2 sub + 1 of atom 7
+        uint4 lo = ld_shared_v4(rrow + kDsv4Nope + 32 * sub);
+        uint4 hi = ld_shared_v4(rrow + kDsv4Nope + 32 * sub + 16);
+        if (!valid) lo = hi = make_uint4(0u, 0u, 0u, 0u);
+        st_shared_v4(tbase + 7 * kAtomBytes + lo_off, lo);
+        st_shared_v4(tbase + 7 * kAtomBytes + hi_off, hi);
       }
       // one proxy fence for the tile: generic stores -> tensor-core reads
       fence_proxy_async_smem();
@@ -902,21 +895,23 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // Each warp instruction covers eight rows, four 16-byte chunks of each
     // (lane = 4 row + chunk): spreading an instruction over many rows keeps
     // more DRAM requests independent, which measured faster on B200 than
-    // whole-row instructions.  Copy warp lw owns the 8-row groups g = lw and
-    // lw + 4 of every tile.  Padding rows read nothing (source size 0).
+    // whole-row instructions.  Copy warp lw owns the 8-row groups
+    // g = lw + kCopyWarps i of every tile.  Padding rows read nothing
+    // (source size 0).
+    constexpr int kGpw = 8 / C::kCopyWarps;          // groups per copy warp
     const int lt = threadIdx.x - 32 * kWarpLoad0;  // 0 .. kCopy-1
     const int lw = lt >> 5;
     const int r8 = lane >> 2, c4 = lane & 3;
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages, rs = t % kRing;
       if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1))) break;  // warp-uniform
-      // this lane's row in groups lw and lw + 4, and, for a bulk group, the
-      // row of lane l < 8
-      int rows[2], brow[2];
+      // this lane's row in each of the warp's groups, and, for a bulk group,
+      // the row of lane l < 8
+      int rows[kGpw], brow[kGpw];
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        rows[gi] = s_row[rs * 64 + 8 * (lw + 4 * gi) + r8];
-        brow[gi] = s_row[rs * 64 + 8 * (lw + 4 * gi) + (lane & 7)];
+      for (int gi = 0; gi < kGpw; ++gi) {
+        rows[gi] = s_row[rs * 64 + 8 * (lw + C::kCopyWarps * gi) + r8];
+        brow[gi] = s_row[rs * 64 + 8 * (lw + C::kCopyWarps * gi) + (lane & 7)];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
@@ -929,8 +924,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         // of a row is 16-byte chunk c % 8 of atom c / 8
         const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
 #pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-          const int tok = 8 * (lw + 4 * gi) + r8;
+        for (int gi = 0; gi < kGpw; ++gi) {
+          const int tok = 8 * (lw + C::kCopyWarps * gi) + r8;
           const int row = rows[gi];
           const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16;
           const uint32_t nbytes = row >= 0 ? 16u : 0u;
@@ -954,8 +949,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
           else return p.kv + (size_t)r * kRowBytesFp8;
         };
 #pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-          const int g = lw + 4 * gi;
+        for (int gi = 0; gi < kGpw; ++gi) {
+          const int g = lw + C::kCopyWarps * gi;
           if (g >= C::kCpGroups) {
             // bulk group: lane l < 8 copies row 8 g + l when it is valid
             const bool v = lane < 8 && brow[gi] >= 0;
