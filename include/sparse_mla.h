@@ -96,9 +96,18 @@ typedef enum {
 } smla_kv_dtype;
 
 /* Problem description.  num_heads must be 64, d_v 512, d_qk 576 (512 for
- * SMLA_KV_DSV4_PAGED). */
+ * SMLA_KV_DSV4_PAGED).
+ *
+ * Multi-token decode (tokens_per_seq = T > 1: speculative / multi-token
+ * prediction steps, where several new tokens of a sequence are scored at
+ * once): every tensor indexed by sequence gains a token dim after it --
+ * q [B, T, 64, d_qk], indices [B, T, topk], out [B, T, 64, 512],
+ * lse [B, T, 64] -- while page_table stays [B, pages_per_seq], shared by the
+ * sequence's tokens.  Token t of sequence b attends over its own list
+ * indices[b, t] exactly as a single decode token does, so each (b, t) row
+ * is one decode problem (B * T rows in all, at most 65535). */
 typedef struct {
-  int32_t batch;          /* B >= 1: sequences, one query token each          */
+  int32_t batch;          /* B >= 1: sequences                                 */
   int32_t num_heads;      /* H = 64                                            */
   int32_t d_qk;           /* 576 = 512 latent + 64 rope (512 for DSV4 pages)   */
   int32_t d_v;            /* 512: the value is the first 512 dims of the row   */
@@ -112,7 +121,8 @@ typedef struct {
   int32_t nsplit;         /* 0: the planner picks the top-k split; >= 1
                              forces that many splits (clamped to the number
                              of 64-entry tiles of the list)                    */
-  int32_t reserved;       /* must be 0                                         */
+  int32_t tokens_per_seq; /* T: query tokens per sequence, 0 or 1 = one token,
+                             at most 16                                        */
 } smla_shape;
 
 /* ABI version of the loaded library (SMLA_ABI_VERSION). */
@@ -130,10 +140,12 @@ const char* sparse_mla_status_string(smla_status status);
  * two ways (sparse_mla_plan_merge tells which).  When nsplit is a power of
  * two no larger than 16 that the device can launch as a thread-block
  * cluster, the CTAs of a sequence form a cluster: each writes its result,
- * normalised by its own softmax sum and rounded to fp16 (11 significant
- * bits; value magnitudes must stay within the fp16 range), to the
- * workspace, the cluster synchronises, and each CTA reduces one block of
- * output columns -- one kernel.  Otherwise each split writes an fp32
+ * normalised by its own softmax sum, to the workspace as fp16 -- each
+ * 128-dim part of a head's row scaled by the power of two that brings its
+ * largest magnitude into [2^14, 2^15), so any finite value fits, with 11
+ * significant bits of that part's largest value -- the cluster
+ * synchronises, and each CTA reduces one block of output columns -- one
+ * kernel.  Otherwise each split writes an fp32
  * partial result and a second (combine) kernel merges them.  An automatic
  * plan (shape->nsplit == 0) takes the largest such power of two for which
  * all clusters are resident at once. */
@@ -153,6 +165,10 @@ size_t sparse_mla_workspace_size(const smla_shape* shape);
 
 /* One decode step: the split kernel, plus the combine kernel when the plan
  * merges its splits through a second kernel (sparse_mla_plan_merge == 2).
+ * (Layouts for one token per sequence; with tokens_per_seq = T > 1 the q,
+ * indices, out and lse tensors carry the extra token dim described at
+ * smla_shape, and B below reads as the B * T decode rows, page_table
+ * excepted.)
  *   q            [B, 64, 576] bf16 ([B, 64, 512] for SMLA_KV_DSV4_PAGED)
  *   kv_cache     [num_kv_rows, 576] bf16, or uint8 e4m3fn codes, or
  *                [num_kv_rows / 64, 37376] uint8 DeepSeek-V4 pages
@@ -220,9 +236,9 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
 /* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:
- * 24 MiB, enough for batch * nsplit <= 191 split results (at most 131,328
- * bytes each).  Every split count the planner picks on a 148-SM B200 fits
- * (it keeps batch * nsplit <= 148). */
+ * 24 MiB, enough for rows * nsplit <= 191 split results (rows = batch x
+ * tokens_per_seq; at most 131,328 bytes each).  Every split count the
+ * planner picks on a 148-SM B200 fits (it keeps rows * nsplit <= 148). */
 #define SMLA_STATIC_SCRATCH_BYTES ((size_t)24 << 20)
 
 /* The whole decode step, for callers that cannot allocate device memory.
@@ -237,7 +253,7 @@ smla_status sparse_mla_get_device_error(uint32_t* code);
  *
  * - Size limit.  A shape whose split results would not fit is rejected
  *   with SMLA_ERR_WORKSPACE before any launch; when shape->nsplit fixes the
- *   split count and even its partials (131,328 bytes per sequence and
+ *   split count and even its partials (131,328 bytes per decode row and
  *   split) cannot fit, before any CUDA call.  Use sparse_mla_decode with
  *   your own workspace for such shapes.
  * - Zeroing.  Every split writes its whole partial (an empty split writes

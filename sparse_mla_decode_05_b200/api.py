@@ -35,7 +35,7 @@ class SmlaShape(ctypes.Structure):
         ("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32), ("d_qk", ctypes.c_int32),
         ("d_v", ctypes.c_int32), ("topk", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
         ("num_kv_rows", ctypes.c_int64), ("page_size", ctypes.c_int32),
-        ("pages_per_seq", ctypes.c_int32), ("nsplit", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("pages_per_seq", ctypes.c_int32), ("nsplit", ctypes.c_int32), ("tokens_per_seq", ctypes.c_int32),
     ]
 
 
@@ -101,10 +101,21 @@ def _stream(device) -> int:
 
 
 def make_shape(batch: int, topk: int, num_kv_rows: int, *, fp8: bool = False, dsv4: bool = False,
-               page_size: int = 0, pages_per_seq: int = 0, nsplit: int = 0) -> SmlaShape:
+               page_size: int = 0, pages_per_seq: int = 0, nsplit: int = 0, tokens_per_seq: int = 0) -> SmlaShape:
     kind = KV_DSV4_PAGED if dsv4 else (KV_FP8_E4M3_ROWSCALE if fp8 else KV_BF16)
     return SmlaShape(batch, H, DSV4_D_QK if dsv4 else D_QK, D_V, topk, kind,
-                     num_kv_rows, page_size, pages_per_seq, nsplit, 0)
+                     num_kv_rows, page_size, pages_per_seq, nsplit, tokens_per_seq)
+
+
+def _tokens(q) -> int:
+    """Query tokens per sequence: q is [B, 64, d] (one) or [B, T, 64, d]."""
+    return q.shape[1] if q.dim() == 4 else 1
+
+
+def _result_shapes(q):
+    """(out, lse) shapes for q [B, (T,) 64, d]."""
+    lead = tuple(q.shape[:-2])
+    return lead + (H, D_V), lead + (H,)
 
 
 def is_dsv4(kv) -> bool:
@@ -113,10 +124,14 @@ def is_dsv4(kv) -> bool:
 
 
 def shape_for(q, kv, indices, *, page_table=None, page_size: int = 0, nsplit: int = 0) -> SmlaShape:
+    """The shape of one call: q [B, 64, d] with indices [B, topk], or q
+    [B, T, 64, d] with indices [B, T, topk] (T query tokens per sequence)."""
     dsv4 = is_dsv4(kv)
-    return make_shape(q.shape[0], indices.shape[1], kv.shape[0] * (64 if dsv4 else 1),
+    T = _tokens(q)
+    return make_shape(q.shape[0], indices.shape[-1], kv.shape[0] * (64 if dsv4 else 1),
                       fp8=(kv.dtype == torch.uint8 and not dsv4), dsv4=dsv4, page_size=page_size,
-                      pages_per_seq=0 if page_table is None else page_table.shape[1], nsplit=nsplit)
+                      pages_per_seq=0 if page_table is None else page_table.shape[1], nsplit=nsplit,
+                      tokens_per_seq=T if T > 1 else 0)
 
 
 def plan_nsplit(shape: SmlaShape) -> int:
@@ -136,13 +151,13 @@ def workspace_size(shape: SmlaShape) -> int:
 def _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size):
     dsv4 = is_dsv4(kv)
     d_qk = DSV4_D_QK if dsv4 else D_QK
-    if q.dtype != torch.bfloat16 or q.dim() != 3 or q.shape[1:] != (H, d_qk):
-        raise ValueError(f"q must be bf16 [B, 64, {d_qk}]")
+    if q.dtype != torch.bfloat16 or q.dim() not in (3, 4) or q.shape[-2:] != (H, d_qk):
+        raise ValueError(f"q must be bf16 [B, 64, {d_qk}] or [B, T, 64, {d_qk}]")
     if not dsv4 and (kv.dim() != 2 or kv.shape[1] != D_QK or kv.dtype not in (torch.bfloat16, torch.uint8)):
         raise ValueError("kv must be [N, 576] bf16 or uint8 (fp8 e4m3fn codes), or uint8 [pages, 37376] "
                          "DeepSeek-V4 pages")
-    if indices.dtype != torch.int32 or indices.dim() != 2 or indices.shape[0] != q.shape[0]:
-        raise ValueError("indices must be int32 [B, topk]")
+    if indices.dtype != torch.int32 or indices.dim() != q.dim() - 1 or indices.shape[:-1] != q.shape[:-2]:
+        raise ValueError("indices must be int32 [B, topk] ([B, T, topk] for q [B, T, 64, d])")
     if dsv4:
         if kv_row_scale is not None:
             raise ValueError("DeepSeek-V4 pages carry their own scales: kv_row_scale must be None")
@@ -165,10 +180,11 @@ def decode(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=None, 
     _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size)
     shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
     dev = q.device
+    o_shape, l_shape = _result_shapes(q)
     if out is None:
-        out = torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
+        out = torch.empty(o_shape, dtype=torch.bfloat16, device=dev)
     if lse is None:
-        lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
+        lse = torch.empty(l_shape, dtype=torch.float32, device=dev)
     ws_bytes = workspace_size(shape)
     if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -209,12 +225,13 @@ def decode_split(q, kv, indices, scale: float, *, kv_row_scale=None, page_table=
     _check_inputs(q, kv, indices, kv_row_scale, page_table, page_size)
     shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
     dev = q.device
+    o_shape, l_shape = _result_shapes(q)
     if out is None:
-        out = torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
+        out = torch.empty(o_shape, dtype=torch.bfloat16, device=dev)
     if lse is None:
-        lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
+        lse = torch.empty(l_shape, dtype=torch.float32, device=dev)
     nplan = plan_nsplit(shape)
-    ws_bytes = partials_size(q.shape[0], nplan) if nplan > 1 else 0
+    ws_bytes = partials_size(q.shape[0] * _tokens(q), nplan) if nplan > 1 else 0
     if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     n = ctypes.c_int32(0)
@@ -284,8 +301,9 @@ class DecodePlan:
         self.nsplit = plan_nsplit(self.shape)
         # the splits merge inside the split kernel (one launch, no combine)
         self.clustered = plan_merge(self.shape) == 1
-        self.out = out if out is not None else torch.empty((q.shape[0], H, D_V), dtype=torch.bfloat16, device=dev)
-        self.lse = lse if lse is not None else torch.empty((q.shape[0], H), dtype=torch.float32, device=dev)
+        o_shape, l_shape = _result_shapes(q)
+        self.out = out if out is not None else torch.empty(o_shape, dtype=torch.bfloat16, device=dev)
+        self.lse = lse if lse is not None else torch.empty(l_shape, dtype=torch.float32, device=dev)
         ws = workspace_size(self.shape)
         self.workspace = workspace if workspace is not None or ws == 0 else \
             torch.empty(ws, dtype=torch.uint8, device=dev)
@@ -297,8 +315,9 @@ class DecodePlan:
                       _ptr(indices), float(scale), _ptr(self.out), _ptr(self.lse), wsp, wsn)
         self._split_args = self._args + (None,)
         if self.nsplit > 1 and not self.clustered:
-            po, pl = partial_views(self.workspace, q.shape[0], self.nsplit)
-            self._combine_args = (q.shape[0], H, D_V, self.nsplit, _ptr(po), _ptr(pl), _ptr(self.out),
+            rows = q.shape[0] * _tokens(q)
+            po, pl = partial_views(self.workspace, rows, self.nsplit)
+            self._combine_args = (rows, H, D_V, self.nsplit, _ptr(po), _ptr(pl), _ptr(self.out),
                                   _ptr(self.lse))
         else:
             self._combine_args = None
@@ -340,17 +359,18 @@ def _check_host_inputs(q_host, kv, indices_host, kv_row_scale, page_table_host, 
     for name, t in (("kv", kv), ("kv_row_scale", kv_row_scale)):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
-    if q_host.dtype != torch.bfloat16 or q_host.dim() != 3 or q_host.shape[1:] != (H, d_qk):
-        raise ValueError(f"q_host must be bf16 [B, 64, {d_qk}]")
-    B = q_host.shape[0]
-    if indices_host.dtype != torch.int32 or indices_host.dim() != 2 or indices_host.shape[0] != B:
-        raise ValueError("indices_host must be int32 [B, topk]")
+    if q_host.dtype != torch.bfloat16 or q_host.dim() not in (3, 4) or q_host.shape[-2:] != (H, d_qk):
+        raise ValueError(f"q_host must be bf16 [B, 64, {d_qk}] or [B, T, 64, {d_qk}]")
+    if (indices_host.dtype != torch.int32 or indices_host.dim() != q_host.dim() - 1
+            or indices_host.shape[:-1] != q_host.shape[:-2]):
+        raise ValueError("indices_host must be int32 [B, topk] ([B, T, topk] for q [B, T, 64, d])")
     if page_size and (page_table_host is None or page_table_host.dtype != torch.int32):
         raise ValueError("paged cache needs int32 page_table_host [B, pages_per_seq]")
-    if out_host.dtype != torch.bfloat16 or tuple(out_host.shape) != (B, H, D_V):
-        raise ValueError("out_host must be bf16 [B, 64, 512]")
-    if lse_host.dtype != torch.float32 or tuple(lse_host.shape) != (B, H):
-        raise ValueError("lse_host must be float32 [B, 64]")
+    o_shape, l_shape = _result_shapes(q_host)
+    if out_host.dtype != torch.bfloat16 or tuple(out_host.shape) != o_shape:
+        raise ValueError("out_host must be bf16 [B, (T,) 64, 512]")
+    if lse_host.dtype != torch.float32 or tuple(lse_host.shape) != l_shape:
+        raise ValueError("lse_host must be float32 [B, (T,) 64]")
 
 
 class HostDecodePlan:
@@ -367,12 +387,12 @@ class HostDecodePlan:
 
     def __init__(self, q_host, kv, indices_host, scale: float, *, kv_row_scale=None, page_table_host=None,
                  page_size: int = 0, nsplit: int = 0, out_host=None, lse_host=None, staging=None):
-        B = q_host.shape[0]
         pin = q_host.is_pinned()
+        o_shape, l_shape = _result_shapes(q_host)
         if out_host is None:
-            out_host = torch.empty((B, H, D_V), dtype=torch.bfloat16, pin_memory=pin)
+            out_host = torch.empty(o_shape, dtype=torch.bfloat16, pin_memory=pin)
         if lse_host is None:
-            lse_host = torch.empty((B, H), dtype=torch.float32, pin_memory=pin)
+            lse_host = torch.empty(l_shape, dtype=torch.float32, pin_memory=pin)
         _check_host_inputs(q_host, kv, indices_host, kv_row_scale, page_table_host, page_size, out_host,
                            lse_host)
         if is_dsv4(kv):

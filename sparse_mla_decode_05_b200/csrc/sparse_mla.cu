@@ -190,7 +190,8 @@ struct SplitParams {
   float* lse;                  // [B, 64]
   float* part_o;               // [B, nsplit, 64, 512]
   float* part_lse;             // [B, nsplit, 64]
-  int batch, topk, nsplit, ntiles_total;
+  int batch, topk, nsplit, ntiles_total;   // batch: decode rows (sequences x tokens)
+  int tok_per_seq;             // query tokens per sequence (row b reads page-table row b / tok_per_seq)
   int cluster;                 // 1: the nsplit CTAs of a sequence form a cluster and reduce on chip
   int page_size, pages_per_seq;
   int num_kv_rows;             // rows in the pool (64 x pages when paged)
@@ -568,13 +569,19 @@ __device__ __forceinline__ void bulk_load_g2s(uint32_t sdst, const void* gsrc, u
                : "memory");
 }
 
+// Merge statistics per (split, head): m, l_pv, l, -, then the inverse fp16
+// scale of each 128-dim part of the split's exchanged row.
+constexpr int kStatFloats = 8;
+
 // In-cluster merge, final step for one thread: head hh, output columns
-// [col0, col0 + 128 / N) (16 / N units of 8 dims).  Split s's fp16 image
-// holds the thread's dims at lane hh % 16 (+16 for dims >= 256) of quarter
-// q, unit u of the half at ((u / 4) * 4 + u % 4) * 32 lanes.  Every split's
-// columns and statistics (m, l_pv) are loaded together, one L2 round trip
-// (with 16 splits the columns follow the weights), then split s is weighted
-// by 2^(m_s - M) l_pv,s and the sum divided by the sum of those weights.
+// [col0, col0 + 128 / N) (16 / N units of 8 dims), all inside the 128-dim
+// part col0 / 128.  Split s's fp16 image holds the thread's dims at lane
+// hh % 16 (+16 for dims >= 256) of quarter q, unit u of the half at
+// ((u / 4) * 4 + u % 4) * 32 lanes, scaled by a power of two that the
+// statistics undo.  Every split's columns and statistics are loaded
+// together, one L2 round trip (with 16 splits the columns follow the
+// weights), then split s is weighted by 2^(m_s - M) l_pv,s and the sum
+// divided by the sum of those weights.
 template <int N>
 __device__ __forceinline__ void merge_tail(const float* wss, const uint4* wso, int q, int lane, int hh, int col0,
                                            __nv_bfloat16* orow) {
@@ -592,12 +599,15 @@ __device__ __forceinline__ void merge_tail(const float* wss, const uint4* wso, i
         x[s * kU + k] = __ldcg(src + (size_t)s * kSplitU + (size_t)((d >> 5) * 4 + ((d >> 3) & 3)) * 32);
       }
   };
-  // statistics [s][h] = (m, l_pv, l, -); the weights need m and l_pv
-  float w[N], lp[N];
+  // statistics [s][h][kStatFloats]; the weights need m, l_pv and the
+  // inverse scale of part col0 / 128
+  float w[N], lp[N], dn[N];
 #pragma unroll
   for (int s = 0; s < N; ++s) {
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(wss + ((size_t)s * 64 + hh) * 4));
+    const float* st = wss + ((size_t)s * 64 + hh) * kStatFloats;
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(st));
     w[s] = v.x; lp[s] = v.y;
+    dn[s] = __ldcg(st + 4 + (col0 >> 7));
   }
   // with 16 splits the columns are loaded after the weights (registers)
   if constexpr (N < 16) load_columns();
@@ -611,6 +621,8 @@ __device__ __forceinline__ void merge_tail(const float* wss, const uint4* wso, i
     Lp += w[s];
   }
   const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
+#pragma unroll
+  for (int s = 0; s < N; ++s) w[s] *= dn[s];                    // undo the exchange scale
   if constexpr (N >= 16) {
     asm volatile("" ::: "memory");
     load_columns();
@@ -742,7 +754,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       long long r = idx;
       if (p.page_size) {
         if (idx >= (long long)p.pages_per_seq * p.page_size) r = -1;
-        else r = (long long)__ldg(p.page_table + (size_t)b * p.pages_per_seq + idx / p.page_size) * p.page_size +
+        else r = (long long)__ldg(p.page_table + (size_t)(b / p.tok_per_seq) * p.pages_per_seq + idx / p.page_size) *
+                     p.page_size +
                  idx % p.page_size;
       }
       if (r < 0 || r >= p.num_kv_rows) {
@@ -1195,8 +1208,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       if (!aborted && half == 0) {
-        float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
-        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * 4) = make_float4(m_run, l_nrm, l_tot, 0.f);
+        float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * kStatFloats;
+        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * kStatFloats) = make_float4(m_run, l_nrm, l_tot, 0.f);
         // for the merge writers: 1 / (rounded-P sum) of head h
         reinterpret_cast<float*>(smem + C::kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
       }
@@ -1284,7 +1297,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     const int upper = warp >> 2;                             // 0: softmax warp, 1: helper warp
     constexpr size_t kSplitU = (size_t)kH * kDv / 8;         // 16-byte units (8 fp16) per split
     uint4* wso = reinterpret_cast<uint4*>(p.part_o) + (size_t)b * n * kSplitU;     // [src][q][c][u][lane]
-    const float* wss = p.part_lse + (size_t)b * n * 64 * 4;  // [src][64][4]: m, l, l_pv
+    float* wss = p.part_lse + (size_t)b * n * 64 * kStatFloats;  // [src][64][8]: m, l_pv, l, -, part scales
     bool failed = merge_failed;
     if (upper) {
       // every PV has completed (the PV issuer's drain barrier: one phase)
@@ -1293,14 +1306,33 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     }
     const bool bad = group_any(failed, 1, 256);
     if (!bad) {
-      // this split's result for the thread's head, normalised by its own
-      // rounded-P sum (a convex combination of value rows) and rounded to
-      // fp16: 11 significant bits, error <= 2^-12 of the largest value
+      // This split's result for the thread's head, normalised by its own
+      // rounded-P sum (a convex combination of value rows), times a power of
+      // two that puts the largest magnitude of the thread's 128 dims (part
+      // 2 half + upper of the row) in [2^14, 2^15), rounded to fp16: any
+      // finite value fits, with 11 significant bits (error <= 2^-12 of the
+      // part's largest value).  The inverse scale goes to the statistics.
       const float sc = reinterpret_cast<const float*>(smem + C::kAuxRow)[16 * q + (lane & 15)];
       uint4* mine = wso + (size_t)split * kSplitU + (size_t)q * (8 * 4 * 32) + lane;
       const uint32_t olanes = (uint32_t)(32 * q + kLaneO) << 16;
       float o[2][32];
       const int c0 = 4 * upper;
+      float mx = 0.f;
+      if (ntiles > 0) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          tmem_ld_16x32bx2_x32_h256(tmem + olanes + 32u * (uint32_t)(c0 + cc), o[0]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) mx = fmaxf(mx, fabsf(o[0][k]));
+        }
+      }
+      mx *= sc;
+      int ex = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127 : 0;   // mx in [2^ex, 2^(ex+1))
+      ex = max(-100, min(ex, 127));
+      const float scw = sc * __uint_as_float((uint32_t)(127 + 14 - ex) << 23);
+      wss[((size_t)split * 64 + 16 * q + (lane & 15)) * kStatFloats + 4 + 2 * (lane >> 4) + upper] =
+          __uint_as_float((uint32_t)(127 - 14 + ex) << 23);
       if (ntiles > 0) {
         tmem_ld_16x32bx2_x32_h256(tmem + olanes + 32u * (uint32_t)c0, o[0]);
         tmem_wait_ld();
@@ -1315,8 +1347,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float* x = &o[cc & 1][8 * u];
-          mine[(c * 4 + u) * 32] = make_uint4(pack_f16x2(x[0] * sc, x[1] * sc), pack_f16x2(x[2] * sc, x[3] * sc),
-                                              pack_f16x2(x[4] * sc, x[5] * sc), pack_f16x2(x[6] * sc, x[7] * sc));
+          mine[(c * 4 + u) * 32] = make_uint4(pack_f16x2(x[0] * scw, x[1] * scw), pack_f16x2(x[2] * scw, x[3] * scw),
+                                              pack_f16x2(x[4] * scw, x[5] * scw), pack_f16x2(x[6] * scw, x[7] * scw));
         }
         if (ntiles > 0 && cc + 1 < 4) tmem_wait_ld();
       }
@@ -1351,7 +1383,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // idle by now and outside the merging warps 0-7, alongside the column
     // merge
     const int hh = 32 * (warp - 8) + lane;
-    const float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * 4;
+    const float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * kStatFloats;
     if (mbar_wait_cluster(BAR(BAR_CS1), 0)) {
       float mv[16], lr[16];
 #pragma unroll
@@ -1359,7 +1391,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         mv[s2] = -INFINITY;
         lr[s2] = 0.f;
         if (s2 < p.nsplit) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * 4));
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(wss + ((size_t)s2 * 64 + hh) * kStatFloats));
           mv[s2] = v.x; lr[s2] = v.z;
         }
       }
@@ -1426,11 +1458,17 @@ __global__ void __launch_bounds__(128) smla_combine_kernel(const float* __restri
 // ============================================================ host side
 static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Query tokens per sequence (0 means one) and decode rows (sequences x tokens).
+static int tokens_of(const smla_shape* s) { return s->tokens_per_seq > 1 ? s->tokens_per_seq : 1; }
+static int rows_of(const smla_shape* s) { return s->batch * tokens_of(s); }
+
 static smla_status validate_shape(const smla_shape* s) {
   if (!s) return SMLA_ERR_INVALID_ARG;
   if (s->batch < 1 || s->batch > 65535 || s->topk < 1 || s->topk > (1 << 24)) return SMLA_ERR_INVALID_ARG;
+  if (s->tokens_per_seq < 0 || s->tokens_per_seq > 16 || (long long)s->batch * tokens_of(s) > 65535)
+    return SMLA_ERR_INVALID_ARG;
   if (s->num_kv_rows < 1 || s->num_kv_rows > 0x7FFFFFFFLL) return SMLA_ERR_INVALID_ARG;
-  if (s->nsplit < 0 || s->reserved != 0) return SMLA_ERR_INVALID_ARG;
+  if (s->nsplit < 0) return SMLA_ERR_INVALID_ARG;
   if (s->kv_dtype != SMLA_KV_BF16 && s->kv_dtype != SMLA_KV_FP8_E4M3_ROWSCALE && s->kv_dtype != SMLA_KV_DSV4_PAGED)
     return SMLA_ERR_UNSUPPORTED;
   const int want_qk = s->kv_dtype == SMLA_KV_DSV4_PAGED ? 512 : kDqk;
@@ -1460,7 +1498,7 @@ static int plan_nsplit_raw(const smla_shape* s, int num_sms) {
   if (s->nsplit > 0) {
     n = s->nsplit;
   } else {
-    n = num_sms > 0 ? num_sms / s->batch : 1;
+    n = num_sms > 0 ? num_sms / rows_of(s) : 1;
   }
   if (n < 1) n = 1;
   if (n > tiles) n = tiles;
@@ -1490,7 +1528,7 @@ static Plan make_plan(const smla_shape* s, int num_sms, const int active[5]) {
   // best split count for every batch and list length tried.
   for (int lg = 4; lg >= 1; --lg) {
     const int c = 1 << lg;
-    if (c <= pl.n && active[lg] >= s->batch) return Plan{c, true};
+    if (c <= pl.n && active[lg] >= rows_of(s)) return Plan{c, true};
   }
   return Plan{1, false};
 }
@@ -1501,12 +1539,12 @@ static size_t partial_bytes(int batch, int nsplit) {
   return ((o + l + 255) / 256) * 256;
 }
 
-// Workspace of an in-cluster merge: every split's normalised result
-// (B * nsplit * 64 * 512 fp16) and its per-head (m, l, l_pv, -) (B * nsplit
-// * 64 * 4 fp32).
+// Workspace of an in-cluster merge: every split's scaled, normalised result
+// (rows * nsplit * 64 * 512 fp16) and its per-head statistics (rows *
+// nsplit * 64 * kStatFloats fp32).
 static size_t cluster_bytes(int batch, int nsplit) {
   const size_t o = (size_t)batch * nsplit * kH * kDv * 2;
-  const size_t st = (size_t)batch * nsplit * kH * 4 * 4;
+  const size_t st = (size_t)batch * nsplit * kH * kStatFloats * 4;
   return ((o + st + 255) / 256) * 256;
 }
 static size_t workspace_bytes_for(int batch, int nsplit, bool cluster) {
@@ -1625,7 +1663,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   const bool cluster = allow_cluster && pl.cluster;
   if (n > 1) {
     if (!workspace || !aligned(workspace, 256)) return SMLA_ERR_WORKSPACE;
-    if (workspace_bytes < workspace_bytes_for(shape->batch, n, cluster)) return SMLA_ERR_WORKSPACE;
+    if (workspace_bytes < workspace_bytes_for(rows_of(shape), n, cluster)) return SMLA_ERR_WORKSPACE;
   }
   SplitParams prm;
   memset(&prm, 0, sizeof(prm));
@@ -1640,9 +1678,10 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.cluster = cluster ? 1 : 0;
   prm.part_o = static_cast<float*>(workspace);
   prm.part_lse = n > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                  (size_t)shape->batch * n * kH * kDv * (cluster ? 2 : 4))
+                                                  (size_t)rows_of(shape) * n * kH * kDv * (cluster ? 2 : 4))
                        : nullptr;
-  prm.batch = shape->batch;
+  prm.batch = rows_of(shape);
+  prm.tok_per_seq = tokens_of(shape);
   prm.topk = shape->topk;
   prm.nsplit = n;
   prm.ntiles_total = (shape->topk + kTile - 1) / kTile;
@@ -1702,11 +1741,11 @@ static size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 static HostStaging host_staging(const smla_shape* s, size_t ws_bytes) {
   HostStaging h;
   size_t off = 0;
-  h.q_bytes = (size_t)s->batch * kH * s->d_qk * 2;
-  h.idx_bytes = (size_t)s->batch * s->topk * 4;
+  h.q_bytes = (size_t)rows_of(s) * kH * s->d_qk * 2;
+  h.idx_bytes = (size_t)rows_of(s) * s->topk * 4;
   h.pt_bytes = s->page_size ? (size_t)s->batch * s->pages_per_seq * 4 : 0;
-  h.out_bytes = (size_t)s->batch * kH * kDv * 2;
-  h.lse_bytes = (size_t)s->batch * kH * 4;
+  h.out_bytes = (size_t)rows_of(s) * kH * kDv * 2;
+  h.lse_bytes = (size_t)rows_of(s) * kH * 4;
   h.ws_bytes = ws_bytes;
   h.q = off;   off += round256(h.q_bytes);
   h.idx = off; off += round256(h.idx_bytes);
@@ -1750,7 +1789,7 @@ int32_t sparse_mla_plan_nsplit(const smla_shape* shape) {
 size_t sparse_mla_workspace_size(const smla_shape* shape) {
   if (smla::validate_shape(shape) != SMLA_OK) return 0;
   const smla::Plan pl = smla::make_plan(shape, smla::device_sm_count(), smla::caps_for(shape).active);
-  return smla::workspace_bytes_for(shape->batch, pl.n, pl.cluster);
+  return smla::workspace_bytes_for(smla::rows_of(shape), pl.n, pl.cluster);
 }
 
 int32_t sparse_mla_plan_merge(const smla_shape* shape) {
@@ -1780,8 +1819,8 @@ smla_status sparse_mla_decode(const smla_shape* shape, const void* q, const void
   if (st != SMLA_OK || n == 1 || cluster) return st;
   const float* po = static_cast<const float*>(workspace);
   const float* pl = reinterpret_cast<const float*>(static_cast<const uint8_t*>(workspace) +
-                                                   (size_t)shape->batch * n * smla::kH * smla::kDv * 4);
-  return smla::run_combine(shape->batch, n, po, pl, out, lse, static_cast<cudaStream_t>(stream));
+                                                   (size_t)smla::rows_of(shape) * n * smla::kH * smla::kDv * 4);
+  return smla::run_combine(smla::rows_of(shape), n, po, pl, out, lse, static_cast<cudaStream_t>(stream));
 }
 
 smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, int32_t nsplit,
@@ -1806,13 +1845,13 @@ smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void
   // nsplit whose partials cannot fit, whichever way they are merged)
   if (shape->nsplit > 0) {
     const int n0 = smla::plan_nsplit_raw(shape, 0);
-    if (n0 > 1 && smla::partial_bytes(shape->batch, n0) > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
+    if (n0 > 1 && smla::partial_bytes(smla::rows_of(shape), n0) > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
   }
   const int sms = smla::device_sm_count();
   if (sms <= 0) return SMLA_ERR_CUDA;
   const smla::Plan pl = smla::make_plan(shape, sms, smla::caps_for(shape).active);
   const int n = pl.n;
-  const size_t need = smla::workspace_bytes_for(shape->batch, n, pl.cluster);
+  const size_t need = smla::workspace_bytes_for(smla::rows_of(shape), n, pl.cluster);
   if (need > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (need > 0) {

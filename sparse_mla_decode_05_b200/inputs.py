@@ -62,7 +62,17 @@ class Workload:
 
     @property
     def topk(self) -> int:
-        return self.indices.shape[1]
+        return self.indices.shape[-1]
+
+    @property
+    def tokens(self) -> int:
+        """Query tokens per sequence (q [B, T, 64, d] for T > 1)."""
+        return self.q.shape[1] if self.q.dim() == 4 else 1
+
+    @property
+    def rows(self) -> int:
+        """Decode rows: sequences x query tokens."""
+        return self.batch * self.tokens
 
     @property
     def kv_format(self) -> str:
@@ -205,6 +215,59 @@ def paged_bf16(B: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: 
                     meta=dict(B=B, rows_per_seq=rows_per_seq, total_pages=total_pages, topk=topk, seed=seed))
 
 
+def _token_lists(rng, B: int, T: int, R: int, topk: int, overlap: float, *, flat: bool) -> np.ndarray:
+    """[B, T, topk] index lists: token 0 takes topk distinct uniform
+    positions of [0, R); token t > 0 keeps round(overlap * topk) of them (a
+    random subset) and draws the rest afresh, distinct within its list.
+    flat: sequence b's positions are offset to rows [b R, (b+1) R)."""
+    idx = np.empty((B, T, topk), dtype=np.int64)
+    keep = int(round(overlap * topk))
+    for b in range(B):
+        first = _distinct(rng, R, topk)
+        idx[b, 0] = first
+        for t in range(1, T):
+            kept = rng.choice(first, size=keep, replace=False)
+            rest_pool = np.setdiff1d(np.arange(R), kept, assume_unique=True)
+            fresh = rest_pool[_distinct(rng, rest_pool.size, topk - keep)]
+            idx[b, t] = rng.permutation(np.concatenate([kept, fresh]))
+        if flat:
+            idx[b] += b * R
+    return idx
+
+
+def multi_token(B: int, T: int, rows_per_seq: int, total_pages: int, topk: int, *, seed: int,
+                fp8: bool = False, paged: bool = True, overlap: float = 0.75,
+                name: str = "multi_token") -> Workload:
+    """Several query tokens per sequence (multi-token / speculative decode),
+    each with its own top-k list.  q [B, T, 64, 576] ~N(0,1) bf16; the cache
+    is a 64-row paged pool (bf16, or fp8 e4m3fn with an amax/448 row scale)
+    with one page table row per sequence, or, with paged=False, a flat pool
+    where sequence b owns rows [b R, (b+1) R).  Token 0 draws topk distinct
+    uniform positions; token t > 0 keeps round(overlap * topk) of token 0's
+    positions (a random subset) and draws the rest afresh, distinct within
+    its list, so that consecutive tokens of a step share most of their
+    rows.  indices [B, T, topk]."""
+    gen = torch.Generator().manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    q = _normal_bf16(gen, (B * T, H, D_QK)).view(B, T, H, D_QK)
+    n_rows = total_pages * 64 if paged else B * rows_per_seq
+    if fp8:
+        kv, scales = _fp8_rows(gen, n_rows)
+    else:
+        kv, scales = _normal_bf16(gen, (n_rows, D_QK)), None
+    pt = None
+    if paged:
+        pps = rows_per_seq // 64
+        if B * pps > total_pages:
+            raise ValueError("not enough pages for distinct page tables")
+        pt = torch.from_numpy(rng.permutation(total_pages)[: B * pps].reshape(B, pps).astype(np.int32))
+    idx = _token_lists(rng, B, T, rows_per_seq, topk, overlap, flat=not paged)
+    return Workload(name=name, q=q, kv=kv, indices=torch.from_numpy(idx.astype(np.int32)),
+                    kv_row_scale=scales, page_table=pt, page_size=64 if paged else 0,
+                    meta=dict(B=B, T=T, rows_per_seq=rows_per_seq, total_pages=total_pages, topk=topk,
+                              seed=seed, overlap=overlap))
+
+
 DSV4_PAGE_BYTES = 64 * 584          # 64 slots of 576 bytes, then 64 scale blocks of 8 bytes
 
 
@@ -322,11 +385,13 @@ CONFIG_DESCRIPTIONS = {
 }
 
 # Workloads beyond the headline set, measured and parity-tested the same way
-EXTRA_NAMES = ("dsv4",)
+EXTRA_NAMES = ("dsv4", "mt2")
 EXTRA_DESCRIPTIONS = {
     "dsv4": "B=32 k=512 DeepSeek-V4 pages (448 fp8 + UE8M0 group scales, 64 bf16 rope), 8192 rows/seq",
+    "mt2": "B=64 x 2 query tokens, k=2048 per token (75% shared), paged(64) fp8 e4m3 + row scale, 8192 rows/seq",
 }
-_BASE_SEEDS = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005, "dsv4": 1006}
+_BASE_SEEDS = {"c1": 1001, "c2": 1002, "c3": 1003, "c4a": 1004, "c4b": 1004, "c5": 1005, "dsv4": 1006,
+               "mt2": 1008}
 
 
 def make_config(name: str, seed: int | None = None) -> Workload:
@@ -347,6 +412,8 @@ def make_config(name: str, seed: int | None = None) -> Workload:
         return paged_fp8(128, 8192, 16384, 2048, seed=s, name="c5")
     if name == "dsv4":
         return paged_dsv4(32, 8192, 4096, 512, seed=s, name="dsv4")
+    if name == "mt2":
+        return multi_token(64, 2, 8192, 16384, 2048, seed=s, fp8=True, overlap=0.75, name="mt2")
     raise KeyError(name)
 
 
@@ -363,6 +430,10 @@ def reindexed(w: Workload, seed: int) -> Workload:
     q_mult = m.get("q_mult", 1.0)
     q = _normal_bf16(gen, tuple(w.q.shape), mult=q_mult)
     idx = np.full((B, topk), -1, dtype=np.int64)
+    if w.tokens > 1:                                  # multi_token: same recipe, new draws
+        idx = _token_lists(rng, B, w.tokens, m["rows_per_seq"], topk, m["overlap"], flat=not w.page_size)
+        return dataclasses.replace(w, q=q, indices=torch.from_numpy(idx.astype(np.int32)),
+                                   meta=dict(m, reindexed_seed=seed))
     if "lens" in m:                                   # flat_varlen
         lens = np.asarray(m["lens"])
         offs = np.concatenate([[0], np.cumsum(lens)[:-1]])
@@ -402,22 +473,33 @@ def shard_seed(name: str, rank: int) -> int | None:
     return _BASE_SEEDS[name] + 100_000 * rank
 
 
+def gathered_row_count(w: Workload) -> int:
+    """Cache rows the step must read at least once: the valid entries of
+    each index list; with several query tokens per sequence, the union of
+    the tokens' lists of a sequence (a row two tokens share is needed from
+    memory once)."""
+    if w.tokens == 1:
+        return w.valid_count()
+    idx = w.indices.numpy()
+    return int(sum(np.unique(idx[b][idx[b] >= 0]).size for b in range(w.batch)))
+
+
 def algorithmic_bytes(w: Workload) -> int:
-    """Bytes the step must move at minimum: valid gathered rows (row bytes,
-    plus the 4-byte row scale for fp8 pools; a DeepSeek-V4 slot's 576 bytes
-    plus its 7 scale bytes), q, out, lse, the index list and the page
-    table.  Padding entries gather nothing."""
-    n_valid = w.valid_count()
+    """Bytes the step must move at minimum: the gathered rows
+    (gathered_row_count; row bytes, plus the 4-byte row scale for fp8 pools;
+    a DeepSeek-V4 slot's 576 bytes plus its 7 scale bytes), q, out, lse,
+    the index lists and the page table.  Padding entries gather nothing."""
+    n_valid = gathered_row_count(w)
     if w.layout == "dsv4":
         row, d_qk = 576 + 7, 512
     else:
         row = D_QK * (1 if w.kv.dtype == torch.uint8 else 2) + (4 if w.kv_row_scale is not None else 0)
         d_qk = D_QK
-    B = w.batch
+    R = w.rows
     b = n_valid * row
-    b += B * H * d_qk * 2          # q
-    b += B * H * w.d_v * 2         # out
-    b += B * H * 4                 # lse
+    b += R * H * d_qk * 2          # q
+    b += R * H * w.d_v * 2         # out
+    b += R * H * 4                 # lse
     b += w.indices.numel() * 4     # indices
     if w.page_table is not None:
         b += w.page_table.numel() * 4
@@ -425,6 +507,6 @@ def algorithmic_bytes(w: Workload) -> int:
 
 
 def algorithmic_flops(w: Workload) -> int:
-    """2*H*(d_qk + d_v) flops per valid (sequence, row): the score and the
-    value contractions."""
-    return int(w.valid_count() * 2 * H * (w.q.shape[2] + w.d_v))
+    """2*H*(d_qk + d_v) flops per valid (decode row, index entry): the
+    score and the value contractions."""
+    return int(w.valid_count() * 2 * H * (w.q.shape[-1] + w.d_v))

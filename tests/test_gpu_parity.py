@@ -164,6 +164,41 @@ def test_cluster_merge_every_size(n, fp8):
     assert torch.all(out[2].float() == 0) and torch.all(torch.isneginf(lse[2]))
 
 
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("n", [2, 16])
+@pytest.mark.parametrize("c", [1e3, 1e6, 1e-3])
+def test_cluster_merge_large_and_small_values(c, n, fp8):
+    """Value rows scaled by c with q scaled by 1/c, so the scores keep their
+    size and out scales by c (|out| ~ 0.25 c with top-2048 lists: ~2.5e5 at
+    c = 1e6, legal bf16 and far beyond the fp16 range).  The in-cluster
+    merge exchanges each split's result as scaled fp16, so out must stay
+    finite and within the usual bar scaled by c (the step is
+    scale-equivariant up to rounding: 2e-2 c on out, 1e-3 on lse)."""
+    if fp8:
+        w = inputs.paged_fp8(2, 4096, 128, 2048, seed=90 + n)
+        w = inputs.Workload(name="fp8_scaled", q=(w.q.float() / c).to(torch.bfloat16), kv=w.kv,
+                            indices=w.indices, kv_row_scale=w.kv_row_scale * c, page_table=w.page_table,
+                            page_size=w.page_size)
+    else:
+        w = inputs.flat_per_seq(2, 8192, 2048, seed=95 + n)
+        w = inputs.Workload(name="bf16_scaled", q=(w.q.float() / c).to(torch.bfloat16),
+                            kv=(w.kv.float() * c).to(torch.bfloat16), indices=w.indices)
+    d = Dev(w)
+    a = api()
+    shape = a.shape_for(d.q, d.kv, d.indices, page_table=d.page_table, page_size=w.page_size, nsplit=n)
+    if n <= 8:
+        assert a.plan_merge(shape) == 1
+    out, lse = d.run(nsplit=n)
+    torch.cuda.synchronize()
+    out_ref, lse_ref = oracle(w)
+    o = out.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(o))
+    assert np.abs(out_ref).max() > 0.1 * c                    # the values really are that large
+    err = np.abs(o - out_ref).max()
+    assert err <= 2e-2 * c, f"c={c} n={n}: out err {err:.3e} > {2e-2 * c:.3e}"
+    assert ref.lse_rel_err(lse.cpu().numpy().astype(np.float64), lse_ref).max() <= 1e-3
+
+
 def test_cluster_merge_counting_exact():
     """On-chip merge over 8 splits recovers the exact set of gathered rows."""
     w, weights, nval = counting_workload(3, 2048, 8192, fp8=False, paged=False, seed=77)
