@@ -235,6 +235,23 @@ smla_status sparse_mla_combine(int32_t batch, int32_t num_heads, int32_t d_v, in
  * the word was zero; SMLA_ERR_CUDA on a copy failure. */
 smla_status sparse_mla_get_device_error(uint32_t* code);
 
+/* Test hook for the bounded waits; the source pages have no counterpart.
+ * Launches the decode kernel for `shape` (SMLA_KV_BF16, flat cache: page
+ * size 0; one CTA per decode row, no workspace) with every pipeline wait
+ * limited to wait_limit_cycles SM clock cycles and the score-MMA warp
+ * waiting on a barrier that nothing arrives on, in place of the staged
+ * query.  So no MMA is issued, every warp's wait runs out, the kernel sets
+ * bit 0 of the device error word, releases its tensor memory and returns;
+ * out and lse are left unwritten.  The context stays usable: the next
+ * sparse_mla_get_device_error returns SMLA_ERR_DEVICE_TIMEOUT, and later
+ * decodes compute as usual.  Arguments as for sparse_mla_decode (q, kv_cache,
+ * indices, out, lse device pointers owned by the caller).  Returns
+ * SMLA_ERR_UNSUPPORTED for other cache kinds or a paged cache,
+ * SMLA_ERR_INVALID_ARG for wait_limit_cycles outside [1000, 4e9]. */
+smla_status sparse_mla_decode_stalled(const smla_shape* shape, const void* q, const void* kv_cache,
+                                      const int32_t* indices, float scale, void* out, float* lse,
+                                      int64_t wait_limit_cycles, void* stream);
+
 /* Size of the scratch buffer that sparse_mla_decode_static_scratch uses:
  * 24 MiB, enough for rows * nsplit <= 191 split results (rows = batch x
  * tokens_per_seq; at most 131,328 bytes each).  Every split count the
@@ -252,10 +269,12 @@ smla_status sparse_mla_get_device_error(uint32_t* code);
  * call nor the library allocates or frees anything.
  *
  * - Size limit.  A shape whose split results would not fit is rejected
- *   with SMLA_ERR_WORKSPACE before any launch; when shape->nsplit fixes the
- *   split count and even its partials (131,328 bytes per decode row and
- *   split) cannot fit, before any CUDA call.  Use sparse_mla_decode with
- *   your own workspace for such shapes.
+ *   with SMLA_ERR_WORKSPACE before any launch.  When shape->nsplit fixes
+ *   the split count and its results cannot fit whichever way they are
+ *   merged (in-cluster merge, possible for a power of two <= 16: 67,584
+ *   bytes per decode row and split; otherwise 131,328), it is rejected
+ *   before any CUDA call.  Use sparse_mla_decode with your own workspace
+ *   for such shapes.
  * - Zeroing.  Every split writes its whole partial (an empty split writes
  *   o = 0, lse = -inf), so nothing in the scratch has to start at zero and
  *   nothing is cleared.

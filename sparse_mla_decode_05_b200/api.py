@@ -75,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.sparse_mla_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.sparse_mla_decode_static_scratch.restype = I32
     lib.sparse_mla_decode_static_scratch.argtypes = [SP, P, P, P, P, P, F32, P, P, P]
+    lib.sparse_mla_decode_stalled.restype = I32
+    lib.sparse_mla_decode_stalled.argtypes = [SP, P, P, P, F32, P, P, ctypes.c_int64, P]
     IP = ctypes.POINTER(IndexerShape)
     lib.sparse_mla_indexer_scores.restype = I32
     lib.sparse_mla_indexer_scores.argtypes = [IP, P, P, P, P, P, P, P]
@@ -272,6 +274,28 @@ def combine(partial_o, partial_lse, out=None, lse=None):
                                 _stream(dev))
     if st != 0:
         raise SmlaError(st, "sparse_mla_combine")
+    return out, lse
+
+
+def decode_stalled(q, kv, indices, scale: float, wait_limit_cycles: int, out=None, lse=None):
+    """sparse_mla_decode_stalled (a test hook): launches the decode kernel
+    on a flat bf16 cache with the score-MMA warp waiting on a barrier that
+    nothing arrives on and every pipeline wait limited to
+    ``wait_limit_cycles``.  Every wait runs out and the kernel sets the
+    device error word's timeout bit; ``out`` and ``lse`` are left
+    unwritten.  Returns (out, lse)."""
+    _check_inputs(q, kv, indices, None, None, 0)
+    shape = shape_for(q, kv, indices)
+    dev = q.device
+    o_shape, l_shape = _result_shapes(q)
+    if out is None:
+        out = torch.empty(o_shape, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(l_shape, dtype=torch.float32, device=dev)
+    st = lib.sparse_mla_decode_stalled(ctypes.byref(shape), _ptr(q), _ptr(kv), _ptr(indices), float(scale),
+                                       _ptr(out), _ptr(lse), int(wait_limit_cycles), _stream(dev))
+    if st != 0:
+        raise SmlaError(st, "sparse_mla_decode_stalled")
     return out, lse
 
 

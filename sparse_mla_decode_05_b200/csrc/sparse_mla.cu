@@ -196,6 +196,8 @@ struct SplitParams {
   int page_size, pages_per_seq;
   int num_kv_rows;             // rows in the pool (64 x pages when paged)
   float scale_log2;            // scale * log2(e)
+  long long wait_limit;        // cycles a pipeline wait may take before it gives up
+  int stall_test;              // 1: the score issuer waits on a barrier nothing arrives on (test of the bounded waits)
 };
 
 __device__ unsigned int g_error_word = 0;
@@ -234,15 +236,16 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false (and an error bit) if the phase did not complete in time.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Bounded wait: false (and an error bit) if the phase did not complete
+// within `limit` SM clock cycles.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_error_word, 1u);
       return false;
     }
@@ -665,6 +668,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // pipeline waits give up after wl cycles (waits on copies and MMAs that
+  // always complete -- the staged query, the MMA drains -- keep the default)
+  const long long wl = p.wait_limit;
   const int split = blockIdx.x;
   const int b = blockIdx.y;
   const int t_begin = (int)((long long)split * p.ntiles_total / p.nsplit);
@@ -809,7 +815,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       }
       const int r2_0 = row_of(i2_0), r2_1 = row_of(i2_1);
       const int i3_0 = idx_at(t + 3 * S, lane), i3_1 = idx_at(t + 3 * S, lane + 32);
-      const bool fail = t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1);
+      const bool fail = t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1, wl);
       if (__any_sync(0xffffffffu, fail)) break;  // warp-uniform exit
       // rows first (the loaders need only them), then the row scales
       s_row[rs * 64 + lane] = r0_0;
@@ -850,16 +856,16 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     const uint32_t lo_off = sw128_off(tok, 2 * sub), hi_off = sw128_off(tok, 2 * sub + 1);
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages, rst = t % kRaw, rs = t % kRing;
-      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXS + rs), (t / kRing) & 1))) break;
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXS + rs), (t / kRing) & 1, wl))) break;
       const bool valid = s_row[rs * 64 + tok] >= 0;
       const uint2 dsc = kDsv4 ? s_dsc[rs * 64 + tok] : make_uint2(0u, 0u);
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + rst), (t / kRaw) & 1))) break;
-      if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_RAW + rst), (t / kRaw) & 1, wl))) break;
+      if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1, wl)))
         break;
       // the last operand stage first holds the staged query
-      if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0))) break;
+      if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0, wl))) break;
       const uint32_t rrow = sbase + C::kSmemRaw + rst * kRawTileBytes + tok * kRawRowBytes;
       const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
       // all loads first (independent), then convert and store
@@ -917,7 +923,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     const int r8 = lane >> 2, c4 = lane & 3;
     for (int t = 0; t < ntiles; ++t) {
       const int stage = t % kStages, rs = t % kRing;
-      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1))) break;  // warp-uniform
+      if (__any_sync(0xffffffffu, !mbar_wait(BAR(BAR_IXF + rs), (t / kRing) & 1, wl))) break;  // warp-uniform
       // this lane's row in each of the warp's groups, and, for a bulk group,
       // the row of lane l < 8
       int rows[kGpw], brow[kGpw];
@@ -929,10 +935,10 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
       if constexpr (!kConv) {
-        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1)))
+        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1, wl)))
           break;
         // the last stage first holds the staged query
-        if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0))) break;
+        if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0, wl))) break;
         // bf16 rows straight into the swizzled operand tile: chunk c (0..71)
         // of a row is 16-byte chunk c % 8 of atom c / 8
         const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
@@ -954,7 +960,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         // g < kCpGroups by cp.async, the others one bulk copy per row
         const int rst = t % C::kRawStages;
         if (__any_sync(0xffffffffu, t >= C::kRawStages &&
-                                        !mbar_wait(BAR(BAR_RAWE + rst), ((t / C::kRawStages) - 1) & 1)))
+                                        !mbar_wait(BAR(BAR_RAWE + rst), ((t / C::kRawStages) - 1) & 1, wl)))
           break;
         const uint32_t rbase = sbase + C::kSmemRaw + rst * kRawTileBytes;
         auto row_src = [&](int r) -> const uint8_t* {
@@ -996,12 +1002,15 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // the issuing thread's own MMAs.  Operand addresses advance by constants
     // (shared descriptors: byte offset >> 4; tensor memory: columns).
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
-      return __shfl_sync(0xffffffffu, (int)mbar_wait(bar, parity), 0) != 0;
+      return __shfl_sync(0xffffffffu, (int)mbar_wait(bar, parity, wl), 0) != 0;
     };
     bool ok = true;
     if (warp == kWarpS) {
       const uint64_t dk0 = sw128_desc(sbase + kSmemKV, 16, 1024);
-      ok = wait_all(BAR(BAR_QT), 0);
+      // (stall_test: the cluster barrier, which nothing arrives on without a
+      // cluster, stands in for the query: the wait runs out, no MMA is
+      // issued, and every other warp's wait runs out in turn)
+      ok = wait_all(BAR(p.stall_test ? BAR_CS1 : BAR_QT), 0);
       tc_fence_after();
       for (int t = 0; ok && t < ntiles; ++t) {
         const int stage = t % kStages, sb = t & 1;
@@ -1100,7 +1109,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     bool aborted = false;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1, rs = i % kRing;
-      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1)) {
+      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1, wl) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1, wl)) {
         aborted = true;
       }
       if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
@@ -1160,7 +1169,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // stage, and PV(i+1) needs this warp's P(i+1).
       const bool resc = need && i >= 1 && m_run > -INFINITY;
       if (__any_sync(0xffffffffu, resc)) {
-        if (!mbar_wait(BAR(BAR_PVD + ((i - 1) & 1)), ((i - 1) >> 1) & 1)) aborted = true;
+        if (!mbar_wait(BAR(BAR_PVD + ((i - 1) & 1)), ((i - 1) >> 1) & 1, wl)) aborted = true;
         if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
         tc_fence_after();
         const float f = resc ? alpha : 1.f;
@@ -1196,8 +1205,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     if (threadIdx.x == 0) grid_dep_launch();
     if (!aborted && ntiles > 0) {
       // PV(n-2) then PV(n-1): each wait is at most one phase ahead
-      if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + (ntiles & 1)), ((ntiles - 2) >> 1) & 1)) aborted = true;
-      if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1)) aborted = true;
+      if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + (ntiles & 1)), ((ntiles - 2) >> 1) & 1, wl)) aborted = true;
+      if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1, wl)) aborted = true;
       aborted = __any_sync(0xffffffffu, aborted);
       tc_fence_after();
     }
@@ -1645,7 +1654,7 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
                              const float* kv_row_scale, const int32_t* page_table, const int32_t* indices,
                              float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                              int32_t* nsplit_out, cudaStream_t stream, int* nsplit_used, bool allow_cluster,
-                             bool* cluster_used) {
+                             bool* cluster_used, long long wait_limit = kWaitLimitCycles, int stall_test = 0) {
   smla_status st = validate_shape(shape);
   if (st != SMLA_OK) return st;
   if (!q || !kv_cache || !indices || !out || !lse) return SMLA_ERR_INVALID_ARG;
@@ -1688,6 +1697,8 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.page_size = shape->page_size;
   prm.pages_per_seq = shape->pages_per_seq;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
+  prm.wait_limit = wait_limit;
+  prm.stall_test = stall_test;
   const cudaError_t e = fp8 ? launch_split<kKindFp8>(prm, stream)
                             : (shape->kv_dtype == SMLA_KV_DSV4_PAGED ? launch_split<kKindDsv4>(prm, stream)
                                                                     : launch_split<kKindBf16>(prm, stream));
@@ -1841,11 +1852,15 @@ smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void
                                              void* stream) {
   smla_status st = smla::validate_shape(shape);
   if (st != SMLA_OK) return st;
-  // split count and scratch need (no CUDA call when the caller fixes an
-  // nsplit whose partials cannot fit, whichever way they are merged)
+  // split count and scratch need.  No CUDA call when the caller fixes an
+  // nsplit whose results fit neither way: the in-cluster merge (possible
+  // for a power of two <= 16, whether the device can launch it or not) needs
+  // the smaller workspace, the separate combine the larger.
   if (shape->nsplit > 0) {
     const int n0 = smla::plan_nsplit_raw(shape, 0);
-    if (n0 > 1 && smla::partial_bytes(smla::rows_of(shape), n0) > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;
+    const bool pow2 = n0 > 1 && (n0 & (n0 - 1)) == 0 && n0 <= 16;
+    if (n0 > 1 && smla::workspace_bytes_for(smla::rows_of(shape), n0, pow2) > SMLA_STATIC_SCRATCH_BYTES)
+      return SMLA_ERR_WORKSPACE;
   }
   const int sms = smla::device_sm_count();
   if (sms <= 0) return SMLA_ERR_CUDA;
@@ -1905,6 +1920,20 @@ smla_status sparse_mla_decode_host(const smla_shape* shape, const void* q_host, 
       cudaMemcpyAsync(lse_host, base + h.lse, h.lse_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return SMLA_ERR_CUDA;
   return SMLA_OK;
+}
+
+smla_status sparse_mla_decode_stalled(const smla_shape* shape, const void* q, const void* kv_cache,
+                                      const int32_t* indices, float scale, void* out, float* lse,
+                                      int64_t wait_limit_cycles, void* stream) {
+  smla_status st = smla::validate_shape(shape);
+  if (st != SMLA_OK) return st;
+  if (shape->kv_dtype != SMLA_KV_BF16 || shape->page_size != 0) return SMLA_ERR_UNSUPPORTED;
+  if (wait_limit_cycles < 1000 || wait_limit_cycles > smla::kWaitLimitCycles) return SMLA_ERR_INVALID_ARG;
+  // one CTA per sequence: no partials, no workspace, no cluster
+  smla_shape one = *shape;
+  one.nsplit = 1;
+  return smla::run_split(&one, q, kv_cache, nullptr, nullptr, indices, scale, out, lse, nullptr, 0, nullptr,
+                         static_cast<cudaStream_t>(stream), nullptr, false, nullptr, (long long)wait_limit_cycles, 1);
 }
 
 smla_status sparse_mla_get_device_error(uint32_t* code) {

@@ -34,7 +34,8 @@ def test_header_declares_the_entry_points():
                  "sparse_mla_workspace_size", "sparse_mla_plan_nsplit", "sparse_mla_status_string",
                  "sparse_mla_abi_version", "sparse_mla_get_device_error", "sparse_mla_plan_merge",
                  "sparse_mla_decode_static_scratch", "sparse_mla_decode_host", "sparse_mla_host_staging_size",
-                 "sparse_mla_indexer", "sparse_mla_indexer_scores", "sparse_mla_indexer_topk"):
+                 "sparse_mla_indexer", "sparse_mla_indexer_scores", "sparse_mla_indexer_topk",
+                 "sparse_mla_decode_stalled"):
         assert must in names
 
 
@@ -241,3 +242,15 @@ def test_indexer_null_and_misaligned_pointers_rejected():
     assert g(ctypes.byref(s), None, 16, 16, None) == INVALID
     assert g(ctypes.byref(s), 16, 16, 2, None) == INVALID
     assert api.lib.sparse_mla_indexer(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, None) == INVALID
+
+
+# ------------------------------------------------ bounded-wait test hook
+def test_stalled_hook_checks_before_any_cuda_call():
+    f = api.lib.sparse_mla_decode_stalled
+    s = shape()
+    assert f(None, 16, 16, 16, 0.04, 16, 16, 100000, None) == INVALID
+    assert f(ctypes.byref(shape(fp8=True)), 16, 16, 16, 0.04, 16, 16, 100000, None) == UNSUPPORTED
+    assert f(ctypes.byref(shape(page_size=64, pages_per_seq=4)), 16, 16, 16, 0.04, 16, 16, 100000,
+             None) == UNSUPPORTED
+    for lim in (-1, 0, 999, 4_000_000_001):
+        assert f(ctypes.byref(s), 16, 16, 16, 0.04, 16, 16, lim, None) == INVALID

@@ -32,6 +32,26 @@ def test_over_the_limit_rejected_before_any_cuda_call(batch, topk, nsplit):
     assert _static(s) == WORKSPACE
 
 
+@pytest.mark.skipif(torch.cuda.is_available(), reason="the shape passes the host checks and would launch")
+@pytest.mark.parametrize("batch,nsplit", [(64, 4), (20, 16)])
+def test_fixed_power_of_two_split_is_not_rejected_when_the_cluster_merge_fits(batch, nsplit):
+    # the separate combine's partials would not fit, the in-cluster merge's
+    # workspace (64 x 512 fp16 + 64 x 8 fp32 per split) does: the host
+    # checks pass it on to the device query, which fails without a GPU
+    assert batch * nsplit * PARTIAL_BYTES > api.STATIC_SCRATCH_BYTES
+    assert batch * nsplit * (64 * 512 * 2 + 64 * 32) <= api.STATIC_SCRATCH_BYTES
+    s = api.make_shape(batch, 64 * nsplit, 100000, nsplit=nsplit)
+    assert _static(s) not in (WORKSPACE, 0)
+
+
+@pytest.mark.parametrize("batch,nsplit", [(8, 32), (16, 24)])
+def test_fixed_split_without_cluster_merge_is_rejected_on_its_partials(batch, nsplit):
+    # more than 16 splits, or not a power of two: only the separate combine
+    assert batch * nsplit * PARTIAL_BYTES > api.STATIC_SCRATCH_BYTES
+    s = api.make_shape(batch, 64 * nsplit, 100000, nsplit=nsplit)
+    assert _static(s) == WORKSPACE
+
+
 def test_limit_constant_matches_header():
     import os
     import re
