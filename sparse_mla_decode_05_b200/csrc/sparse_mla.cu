@@ -80,12 +80,17 @@ constexpr int kRawTileBytes = kTile * kRawRowBytes; // 36,864
 // holds tile t: S(t) has read that atom by the time P(t) is written, PV(t)
 // reads the rest of the stage, and the stage is refilled only after PV(t).
 // Each stage thus carries its own P buffer.
-// Raw stage (fp8 / DeepSeek-V4 caches): one tile's rows as stored, 576
+// Raw stage (DeepSeek-V4 caches): one tile's rows as stored, 576
 // contiguous bytes per row, before conversion to bf16.
+// fp8 caches compute on the codes as stored: an operand stage is one tile
+// of 576-code rows as 8-row x 16-byte core matrices (no swizzle; K-major
+// for S, MN-major for PV), and P(t) goes to one of two separate P buffers
+// ([64 heads][128 codes: 64 tokens high part, 64 low part], 128-byte
+// swizzled, K-major).
 constexpr int kSmemKV = 0;
 constexpr int kAtomP = kAtoms - 1;
 constexpr int kRing = 4;                            // resolved-row ring depth (tiles)
-constexpr int kMaxStages = 3;
+constexpr int kMaxStages = 5;
 // barrier indices
 constexpr int BAR_KVF = 0;                          // [stages] operand tile ready
 constexpr int BAR_KVE = BAR_KVF + kMaxStages;       // [stages] operand tile consumed (PV done)
@@ -97,8 +102,7 @@ constexpr int BAR_FIN = BAR_PVD + 2;                // drain, S issuer
 constexpr int BAR_FIN2 = BAR_FIN + 1;               // drain, PV issuer
 constexpr int BAR_QT = BAR_FIN2 + 1;                // query written to TMEM
 constexpr int BAR_QS = BAR_QT + 1;                  // query staged in shared memory
-constexpr int BAR_PVI = BAR_QS + 1;                 // [2] PV(t) issued (by tile parity)
-constexpr int BAR_IXF = BAR_PVI + 2;                // [kRing] rows resolved
+constexpr int BAR_IXF = BAR_QS + 1;                 // [kRing] rows resolved
 constexpr int BAR_IXS = BAR_IXF + kRing;            // [kRing] row scales / scale blocks resolved
 constexpr int BAR_IXE = BAR_IXS + kRing;            // [kRing] rows consumed
 constexpr int BAR_RAW = BAR_IXE + kRing;            // [raw stages] raw rows landed
@@ -134,27 +138,39 @@ constexpr uint32_t make_idesc(int M, int N, bool a_mn_major, bool b_mn_major) {
 }
 constexpr uint32_t kIdescS = make_idesc(64, 64, false, false);    // S = Q K^T   (Q from TMEM)
 constexpr uint32_t kIdescPV = make_idesc(64, 256, false, true);   // O += P V    (V MN-major)
+// Instruction descriptors (kind::f8f6f4): D f32, A and B e4m3 (format 0 in
+// bits 7-9 and 10-12), B major bit 16, N>>3 at 17, M>>4 at 24.
+constexpr uint32_t make_idesc_e4m3(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+constexpr uint32_t kIdescS8 = make_idesc_e4m3(64, 64, false);    // S = [Qhi | Qlo] [K; K]^T
+constexpr uint32_t kIdescPV8 = make_idesc_e4m3(64, 256, true);   // O += [Phi | Plo] [V; V]
 
 // Bounded waits give up after this many SM clock cycles (about 2 s).
 constexpr long long kWaitLimitCycles = 4000000000ll;
 
-// warps 0-3 softmax/epilogue, 4 S-MMA issuer (+ TMEM allocator), 5 PV-MMA
-// issuer, 6-9 index resolvers (warp 6+k owns the tiles t = k mod 4), 10-13
-// copy warps, then, for fp8 and DeepSeek-V4 caches, four warps that convert
-// the raw codes to bf16 operand tiles
-constexpr int kWarpS = 4, kWarpPV = 5, kWarpIdx = 6, kIdxWarps = 4, kWarpLoad0 = kWarpIdx + kIdxWarps;
-// the in-cluster merge uses warps 0-7 and, for the lse, index warps 8-9
-static_assert(kWarpIdx <= 8 && kWarpIdx + kIdxWarps >= 10, "warps 8 and 9 must be index warps");
+// Warp roles: S softmax/epilogue warps (two per tensor-memory lane quarter,
+// or one for DeepSeek-V4 caches), then the S-MMA issuer (+ TMEM allocator),
+// the PV-MMA issuer, four index resolvers (resolver k owns the tiles t = k
+// mod 4), the copy warps and, for DeepSeek-V4 caches, eight warps that
+// convert the raw codes to bf16 operand tiles.  The in-cluster merge uses
+// warps 0-7 and, for the lse, warps 8-9, all done with their roles by then.
+constexpr int kIdxWarps = 4;
 // cache layouts the split kernel is instantiated for
 constexpr int kKindBf16 = 0;   // bf16 rows [N, 576]
 constexpr int kKindFp8 = 1;    // e4m3fn rows [N, 576] + one fp32 scale per row
 constexpr int kKindDsv4 = 2;   // DeepSeek-V4 pages: 448 e4m3fn + UE8M0 group scales, 64 bf16 rope
 template <int kKind>
 struct Cfg {
-  static constexpr bool kConv = kKind != kKindBf16;     // raw codes converted to bf16 by convert warps
-  static constexpr int kStages = kConv ? 2 : 3;         // operand stages
+  static constexpr bool kNat = kKind == kKindFp8;       // e4m3 MMAs on the codes as stored
+  static constexpr bool kConv = kKind == kKindDsv4;     // raw codes converted to bf16 by convert warps
+  static constexpr int kStages = kNat ? 5 : (kConv ? 2 : 3);   // operand stages
+  static constexpr int kOpBytes = kNat ? kRawTileBytes : kTileBytes;   // bytes per operand stage
   static constexpr int kRawStages = kConv ? 2 : 0;      // raw stages
-  static constexpr int kQStage = kStages - 1;           // holds the staged query until it is in TMEM
+  static constexpr int kQStage = kStages - 1;           // holds the staged query until it is in TMEM (bf16 operands)
+  static constexpr int kSmxWarps = kConv ? 4 : 8;
+  static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + 1, kWarpIdx = kSmxWarps + 2;
+  static constexpr int kWarpLoad0 = kWarpIdx + kIdxWarps;
   static constexpr int kCopyWarps = kConv ? 2 : 4;
   static constexpr int kCvtWarps = kConv ? 8 : 0;
   static constexpr int kCopyThreads = kCopyWarps * 32;
@@ -166,18 +182,25 @@ struct Cfg {
   static constexpr int kCpGroups = kConv ? 5 : 8;
   static constexpr int kBulkGroups = 8 - kCpGroups;      // one expect-tx arrival each
   // shared memory map
-  static constexpr int kSmemRaw = kSmemKV + kStages * kTileBytes;
+  static constexpr int kSmemP = kSmemKV + kStages * kOpBytes;             // fp8: two P buffers
+  static constexpr int kSmemRaw = kSmemP + (kNat ? 2 * kAtomBytes : 0);
   static constexpr int kSmemAux = kSmemRaw + kRawStages * kRawTileBytes;
   static constexpr int kAuxBars = kSmemAux;
   static constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
   static constexpr int kAuxRow = kAuxTmem + 16;              // int  [kRing][64] physical row or -1
   static constexpr int kAuxRsc = kAuxRow + kRing * 64 * 4;   // f32  [kRing][64] fp8 row scales
   static constexpr int kAuxDsc = kAuxRsc + kRing * 64 * 4;   // u64  [kRing][64] DeepSeek-V4 scale blocks
-  static constexpr int kSmemBytes = kAuxDsc + kRing * 64 * 8;
+  static constexpr int kAuxXch = kAuxDsc + kRing * 64 * 8;   // f32  [2][2][64] softmax exchange
+  static constexpr int kAuxQsc = kAuxXch + 2 * 2 * 64 * 4;   // f32  [64] fp8 query scales
+  static constexpr int kSmemBytes = kAuxQsc + 64 * 4;
   static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
   static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxDsc % 16 == 0, "aux arrays are read as vectors");
   static_assert(8 % kCopyWarps == 0 && kCpGroups >= 1 && kCpGroups <= 8, "copy-warp group ownership");
   static_assert(!kConv || kCvtWarps == 8, "convert warps: one thread per (row, 16-code column)");
+  static_assert(kSmemP % 1024 == 0, "P buffers are 128-byte swizzled (1024-byte aligned)");
+  static_assert(kStages <= kMaxStages, "barrier arrays");
+  static_assert(kSmxWarps == 4 || kSmxWarps == 8, "one or two softmax warps per lane quarter");
+  static_assert(kWarpLoad0 >= 10, "warps 8 and 9 exist beside the merging warps 0-7");
 };
 
 struct SplitParams {
@@ -237,9 +260,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Bounded wait: false (and an error bit) if the phase did not complete
-// within `limit` SM clock cycles.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
-  if (mbar_try_wait(bar, parity)) return true;
+// within `limit` SM clock cycles.  The first probe is inline; the loop is
+// out of line.
+__device__ __noinline__ bool mbar_wait_loop(uint32_t bar, uint32_t parity, long long limit) {
   const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
@@ -250,6 +273,9 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long 
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit = kWaitLimitCycles) {
+  return mbar_try_wait(bar, parity) || mbar_wait_loop(bar, parity, limit);
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
@@ -344,6 +370,46 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4_scaled(uint32_t w, uint32_t s2,
   lo = bf16x2_mul(lo, s2);
   hi = bf16x2_mul(hi, s2);
 }
+// Two fp32 -> packed e4m3x2 (lo in the low byte), round to nearest even,
+// saturating at +-448.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// packed e4m3x2 (low byte first) -> two fp32, exact
+__device__ __forceinline__ float2 unpack_e4m3x2(uint32_t v) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)v));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+// x = hi + lo with hi = e4m3(x) and lo = e4m3(x - hi): exact for a bf16 x
+// (8 significant bits) whose parts are e4m3 normals, and within half an
+// e4m3 subnormal step (2^-10) otherwise.  Returns hi and lo as e4m3x2
+// pairs for (x0, x1).
+__device__ __forceinline__ void split_e4m3x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = pack_e4m3x2(x0, x1);
+  const float2 h = unpack_e4m3x2(hi);
+  lo = pack_e4m3x2(x0 - h.x, x1 - h.y);
+}
+// The same split through f16x2: x is rounded to f16 first (11 significant
+// bits, relative error <= 2^-12), then hi = e4m3(x16), lo = e4m3(x16 - hi)
+// (the difference is exact in f16).  For x in [0, 448).
+__device__ __forceinline__ void split_e4m3x2_h(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t x16 = pack_f16x2(x0, x1);
+  uint16_t h, l;
+  uint32_t h16, r16;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(h) : "r"(x16));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h16) : "h"(h));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r16) : "r"(x16), "r"(h16));
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(l) : "r"(r16));
+  hi = h;
+  lo = l;
+}
+// 2^k for an integer k in [-126, 127]
+__device__ __forceinline__ float pow2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+// floor(log2(x)) for a normal positive x
+__device__ __forceinline__ int ilog2f(float x) { return (int)((__float_as_uint(x) >> 23) & 0xFFu) - 127; }
 // UE8M0 exponent byte e (OCP microscaling E8M0) -> 2^(e - 127) as a bf16x2
 // pair: the byte is the bf16 exponent field, except e = 0 (2^-127, a bf16
 // subnormal) and e = 255 (E8M0 NaN; reads as infinity here).
@@ -410,6 +476,28 @@ __device__ __forceinline__ void mma_ts_acc_elect(uint32_t d_tmem, uint32_t a_tme
       "r"(a_tmem), "l"(b_desc), "r"(idesc)
       : "memory");
 }
+// kind::f8f6f4 (e4m3 x e4m3, fp32 accumulate): A from tensor memory (S) or
+// shared memory (PV)
+__device__ __forceinline__ void mma8_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma8_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)acc)
+      : "memory");
+}
 __device__ __forceinline__ void commit_elect(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -436,6 +524,19 @@ __device__ __forceinline__ void tmem_ld_16x32bx2_x32(uint32_t taddr, float (&v)[
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 lanes x 16 columns, twice: threads 0-15 read columns [c, c+16) of
+// lanes base+0..15, threads 16-31 read columns [c+32, c+48) of the same lanes.
+__device__ __forceinline__ void tmem_ld_16x32bx2_x16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 32;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 // 16 lanes x 32 columns, twice: threads 0-15 access columns [c, c+32) of
 // lanes base+0..15, threads 16-31 columns [c+256, c+288) of the same lanes.
@@ -486,6 +587,31 @@ __device__ __forceinline__ void tmem_st_16x32bx2_x16(uint32_t taddr, const uint3
       "n"(kSplit)
       : "memory");
 }
+
+// 16 lanes x 8 columns, twice: threads 0-15 write columns [c, c+8) of lanes
+// base+0..15, threads 16-31 columns [c+kSplit, c+kSplit+8).
+template <int kSplit>
+__device__ __forceinline__ void tmem_st_16x32bx2_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], %9, {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+      "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "n"(kSplit)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor without swizzle (layout type 0): 8-row x
+// 16-byte core matrices of 128 contiguous bytes.  K-major operand: lbo =
+// the next 16 bytes along K, sbo = the next 8 rows; MN-major operand: lbo
+// = the next 8 rows along K, sbo = the next 16 bytes along MN.
+__device__ __forceinline__ uint64_t cm_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// byte offset of 16-byte chunk c (0..35) of row r in a tile of 576-byte
+// rows held as core matrices: [8-row group][chunk][row in group][16 B]
+__device__ __forceinline__ uint32_t cm_off(int r, int c) {
+  return (uint32_t)(((r >> 3) * (kRawRowBytes / 16) + c) * 128 + (r & 7) * 16);
+}
+constexpr uint32_t kCmGroupBytes = (kRawRowBytes / 16) * 128;   // 4,608: next 8 rows
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start
 // address, leading/stride byte offsets >> 4, version 1 at bit 46, layout
@@ -659,6 +785,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
   constexpr bool kFp8 = kKind == kKindFp8;     // row scale folded into S and P
   constexpr bool kDsv4 = kKind == kKindDsv4;
   constexpr bool kConv = C::kConv;
+  constexpr bool kNat = C::kNat;               // fp8 codes straight into e4m3 MMAs
+  constexpr int kSmx = C::kSmxWarps;
+  constexpr int kWarpS = C::kWarpS, kWarpPV = C::kWarpPV, kWarpIdx = C::kWarpIdx, kWarpLoad0 = C::kWarpLoad0;
   constexpr int kStages = C::kStages;
   constexpr int kQK = kDsv4 ? 512 : kDqk;      // query / key width
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -698,7 +827,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // DeepSeek-V4: one per convert warp
       mbar_init(BAR(BAR_KVF + s), kConv ? C::kCvtWarps : kCopy);
       mbar_init(BAR(BAR_KVE + s), 1);
-      mbar_init(BAR(BAR_PF + s), 4);
+      mbar_init(BAR(BAR_PF + s), kSmx);
     }
     for (int s = 0; s < C::kRawStages; ++s) {
       // one arrival per copying thread when its cp.async land, plus one
@@ -708,9 +837,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(BAR_SF + s), 1);
-      mbar_init(BAR(BAR_SE + s), 4);
+      mbar_init(BAR(BAR_SE + s), kSmx);
       mbar_init(BAR(BAR_PVD + s), 1);
-      mbar_init(BAR(BAR_PVI + s), 1);
     }
     mbar_init(BAR(BAR_FIN), 1);
     mbar_init(BAR(BAR_FIN2), 1);
@@ -722,7 +850,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       mbar_init(BAR(BAR_IXS + r), 1);
       // consumers of a ring slot: the copy warps (rows), the softmax warps
       // (row scales) and the convert warps (rows to zero, scale blocks)
-      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + 4 + C::kCvtWarps);
+      mbar_init(BAR(BAR_IXE + r), kCopy / 32 + kSmx + C::kCvtWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -773,7 +901,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     const int kw = warp - kWarpIdx;
     // the 64 x kQK query (contiguous bf16) into the last operand stage,
     // which no tile uses before the query has been moved to tensor memory
-    if (kw == 0 && lane == 0) {
+    if (!kNat && kw == 0 && lane == 0) {
       constexpr uint32_t kQBytes = (uint32_t)kH * kQK * 2;
       mbar_arrive_expect_tx(BAR(BAR_QS), kQBytes);
       bulk_load_g2s(sbase + kSmemKV + C::kQStage * kTileBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
@@ -934,7 +1062,26 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-      if constexpr (!kConv) {
+      if constexpr (kNat) {
+        if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1, wl)))
+          break;
+        // fp8 rows as stored, into the core-matrix layout: chunk c (0..35)
+        // of a row to cm_off(row in tile, c)
+        const uint32_t tbase = sbase + kSmemKV + stage * C::kOpBytes;
+#pragma unroll
+        for (int gi = 0; gi < kGpw; ++gi) {
+          const int tok = 8 * (lw + C::kCopyWarps * gi) + r8;
+          const int row = rows[gi];
+          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8;
+          const uint32_t nbytes = row >= 0 ? 16u : 0u;
+#pragma unroll
+          for (int sg = 0; sg < 9; ++sg) {
+            const int c = 4 * sg + c4;
+            cp_async_16(tbase + cm_off(tok, c), src + c * 16, nbytes);
+          }
+        }
+        cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
+      } else if constexpr (!kConv) {
         if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1, wl)))
           break;
         // the last stage first holds the staged query
@@ -1015,26 +1162,38 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       for (int t = 0; ok && t < ntiles; ++t) {
         const int stage = t % kStages, sb = t & 1;
         // S(t) reuses the S buffer of S(t-2): its softmax must have read it.
-        // It also waits until PV(t-2) has been issued, which keeps the
-        // tensor-core queue in the order S(t-1), PV(t-2), S(t), PV(t-1):
-        // issued earlier, S(t) would delay PV(t-2) and with it the softmax.
+        // (Nothing else orders S(t) after PV(t-2): issued as soon as the
+        // softmax has read S(t-2), S(t) is done by the time the softmax
+        // reaches tile t, which measured faster than holding it behind
+        // PV(t-2).)
         if (t >= 2) {
-          ok = wait_all(BAR(BAR_SE + sb), ((t >> 1) - 1) & 1) && wait_all(BAR(BAR_PVI + sb), ((t >> 1) - 1) & 1);
+          ok = wait_all(BAR(BAR_SE + sb), ((t >> 1) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
         }
         ok = wait_all(BAR(BAR_KVF + stage), (t / kStages) & 1);
         if (!ok) break;
-        // stage s starts s * kTileBytes later (descriptor address field: bytes >> 4)
-        const uint64_t bk = dk0 + (uint64_t)(stage * (kTileBytes >> 4));
         const uint32_t d = tmem + kColS + 64u * (uint32_t)sb;
-        // 36 K steps: Q columns +8 per step (16 bf16); K descriptor: atom
-        // +512, 16-element step +2
-        mma_ts_set_elect(d, tmem + kColQ, bk, kIdescS);
+        if constexpr (kNat) {
+          // 36 K steps of 32 codes: the query's high part (steps 0-17), then
+          // its low part (18-35), each against K chunks 2 (k mod 18) and +1
+          // (+256 B, +16 in the descriptor); Q columns +8 per step
+          const uint64_t bk = cm_desc(sbase + kSmemKV + stage * C::kOpBytes, 128, kCmGroupBytes);
+          mma8_ts_elect(d, tmem + kColQ, bk, kIdescS8, false);
 #pragma unroll
-        for (int k = 1; k < kQK / 16; ++k) {
-          const uint64_t off = (uint64_t)((k >> 2) * (kAtomBytes >> 4) + (k & 3) * 2);
-          mma_ts_acc_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + off, kIdescS);
+          for (int k = 1; k < 2 * kDqk / 32; ++k)
+            mma8_ts_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + (uint64_t)((k % 18) * 16), kIdescS8, true);
+        } else {
+          // stage s starts s * kTileBytes later (descriptor address field: bytes >> 4)
+          const uint64_t bk = dk0 + (uint64_t)(stage * (kTileBytes >> 4));
+          // 36 K steps: Q columns +8 per step (16 bf16); K descriptor: atom
+          // +512, 16-element step +2
+          mma_ts_set_elect(d, tmem + kColQ, bk, kIdescS);
+#pragma unroll
+          for (int k = 1; k < kQK / 16; ++k) {
+            const uint64_t off = (uint64_t)((k >> 2) * (kAtomBytes >> 4) + (k & 3) * 2);
+            mma_ts_acc_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + off, kIdescS);
+          }
         }
         commit_elect(BAR(BAR_SF + sb));
       }
@@ -1046,42 +1205,143 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         ok = wait_all(BAR(BAR_PF + stage), (t / kStages) & 1);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t bv = dv0 + (uint64_t)(stage * (kTileBytes >> 4));
-        // P(t) sits in the stage's rope atom
-        const uint64_t dp = sw128_desc(sbase + kSmemKV + stage * kTileBytes + kAtomP * kAtomBytes, 16, 1024);
-        // O[:, 256 hf + n] += P[:, 16 kk + k] V[16 kk + k, 256 hf + n]:
-        // A = P (K step +32 B), B = V MN-major (tokens +2048 B, dims 256
-        // = four atoms = +32768 B)
+        if constexpr (kNat) {
+          // O[:, 256 hf + n] += P8[:, 32 kk + k] V[32 (kk mod 2) + k, 256 hf + n]:
+          // A = P buffer t mod 2 (codes 0-63: high parts of the 64 tokens,
+          // 64-127: low parts; K step +32 B), B = the stage's codes
+          // MN-major (8-token groups 4608 B apart, 16-dim chunks 128 B
+          // apart; dims 256 hf = chunk 16 hf)
+          const uint32_t vb = sbase + kSmemKV + stage * C::kOpBytes;
+          const uint64_t dp = sw128_desc(sbase + C::kSmemP + (t & 1) * kAtomBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t d = o0 + 256u * (uint32_t)hf;
-            const uint64_t a = dp + (uint64_t)(2 * kk);
-            const uint64_t bb = bv + (uint64_t)(128 * kk + 2048 * hf);
-            if (t == 0 && kk == 0) mma_set_elect(d, a, bb, kIdescPV);
-            else mma_acc_elect(d, a, bb, kIdescPV);
+            for (int hf = 0; hf < 2; ++hf) {
+              const uint64_t bb = cm_desc(vb + (uint32_t)(((4 * (kk & 1)) * (kRawRowBytes / 16) + 16 * hf) * 128),
+                                          kCmGroupBytes, 128);
+              mma8_ss_elect(o0 + 256u * (uint32_t)hf, dp + (uint64_t)(2 * kk), bb, kIdescPV8, t > 0 || kk > 0);
+            }
+          }
+        } else {
+          const uint64_t bv = dv0 + (uint64_t)(stage * (kTileBytes >> 4));
+          // P(t) sits in the stage's rope atom
+          const uint64_t dp = sw128_desc(sbase + kSmemKV + stage * kTileBytes + kAtomP * kAtomBytes, 16, 1024);
+          // O[:, 256 hf + n] += P[:, 16 kk + k] V[16 kk + k, 256 hf + n]:
+          // A = P (K step +32 B), B = V MN-major (tokens +2048 B, dims 256
+          // = four atoms = +32768 B)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const uint32_t d = o0 + 256u * (uint32_t)hf;
+              const uint64_t a = dp + (uint64_t)(2 * kk);
+              const uint64_t bb = bv + (uint64_t)(128 * kk + 2048 * hf);
+              if (t == 0 && kk == 0) mma_set_elect(d, a, bb, kIdescPV);
+              else mma_acc_elect(d, a, bb, kIdescPV);
+            }
           }
         }
         commit_elect(BAR(BAR_KVE + stage));
         commit_elect(BAR(BAR_PVD + (t & 1)));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_PVI + (t & 1)));
       }
     }
     // drain: every MMA this warp issued has completed before teardown
     commit_elect(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2));
     mbar_wait(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2), 0);
-  } else {
+  } else if (warp < kSmx) {
     // ------------------------------------------------------------ softmax
-    // Thread (warp w, lane t) owns head h = 16w + t%16; lanes t and t+16 hold
-    // tokens [0,32) and [32,64) of a tile and dims [0,256) / [256,512) of O.
-    const int h = 16 * warp + (lane & 15);
+    // kSmx warps; warp w reaches tensor-memory lane quarter q = w % 4 (heads
+    // 16 q .. 16 q + 15).  Thread (w, lane) owns head h = 16 q + lane % 16
+    // and, of every tile, the kTok tokens [32 half + kTok u, +kTok) (half =
+    // lane / 16, u = w / 4); of O it holds dims [256 half, +256), 32-dim
+    // chunks [kOc u, kOc u + kOc).  With two warps per quarter a head's
+    // maxima and sums are combined through shared memory at a barrier of
+    // the softmax warps, which also ORs their abort flags: every softmax
+    // warp leaves the tile loop at the same tile.
+    constexpr int kU = kSmx / 4, kTok = 32 / kU, kOc = 8 / kU;
+    const int q = warp & 3, u = warp >> 2;
+    const int h = 16 * q + (lane & 15);
     const int half = lane >> 4;
-    const uint32_t q_lanes = (uint32_t)(32 * warp) << 16;            // Q / S rows
-    const uint32_t o_lanes = (uint32_t)(32 * warp + kLaneO) << 16;   // O rows
-    {  // the query row into tensor memory: dims [kQK/2 half, +kQK/2), read
-       // from the copy staged in shared memory (row-major [64][kQK])
+    const int tok0 = 32 * half + kTok * u;
+    const uint32_t q_lanes = (uint32_t)(32 * q) << 16;            // Q / S rows
+    const uint32_t o_lanes = (uint32_t)(32 * q + kLaneO) << 16;   // O rows
+    float* s_xch = reinterpret_cast<float*>(smem + C::kAuxXch);   // [2 slots][kU][64]
+    int xc = 0;                                                   // exchanges so far
+    // v combined over the kU warps of head h (max or sum; v already
+    // combined over the thread's two halves), abort flags ORed
+    auto pair_reduce = [&](float v, bool is_max, bool& ab) -> float {
+      if constexpr (kU == 1) {
+        ab = __any_sync(0xffffffffu, ab);
+        return v;
+      } else {
+        float* x = s_xch + (xc & 1) * (2 * 64);
+        ++xc;
+        if (lane < 16) x[u * 64 + h] = v;
+        ab = group_any(ab, 2, 32 * kSmx);
+        const float o = x[(1 - u) * 64 + h];
+        return is_max ? fmaxf(v, o) : v + o;
+      }
+    };
+    // fp8: 2^-sq, the power of two the head's query was scaled by
+    float q_unscale = 1.f;
+    bool aborted = false;
+    if constexpr (kNat) {
+      float* s_qsc = reinterpret_cast<float*>(smem + C::kAuxQsc);
+      if (u == 0) {
+        // The query row as e4m3 parts in tensor memory: x = q * 2^sq (the
+        // head's largest |q| scaled into [128, 256)), high part e4m3(x) at
+        // columns [0, 144), low part e4m3(x - high) at [144, 288); this
+        // thread's dims [288 half, +288) are columns [72 half, +72) of each.
+        // Read straight from global memory, twice (the scale first).
+        const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((size_t)b * kH + h) * (kDqk * 2) + half * kDqk);
+        uint32_t amax = 0;   // largest |q| as bf16 magnitude bits (ordered like the values)
+#pragma unroll 4
+        for (int k4 = 0; k4 < kDqk / 16; ++k4) {
+          const uint4 v = __ldg(qg + k4);
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) amax = max(amax, max(w4[k] & 0x7FFFu, (w4[k] >> 16) & 0x7FFFu));
+        }
+        amax = max(amax, (uint32_t)__shfl_xor_sync(0xffffffffu, (int)amax, 16));
+        const float qmax = __uint_as_float(amax << 16);
+        const int sq = qmax > 0.f ? min(126, max(-126, 7 - ilog2f(qmax))) : 0;   // (subnormal maxima: 126)
+        const float qscale = pow2i(sq);
+        q_unscale = pow2i(-sq);
+#pragma unroll 1
+        for (int c = 0; c < kDqk / 64; ++c) {   // 32 dims per step
+          uint32_t hw[8], lw[8];
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint4 v = __ldg(qg + 4 * c + k4);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; k += 2) {
+              uint32_t h0, l0, h1, l1;
+              split_e4m3x2(__uint_as_float(w4[k] << 16) * qscale, __uint_as_float(w4[k] & 0xFFFF0000u) * qscale,
+                           h0, l0);
+              split_e4m3x2(__uint_as_float(w4[k + 1] << 16) * qscale,
+                           __uint_as_float(w4[k + 1] & 0xFFFF0000u) * qscale, h1, l1);
+              hw[2 * k4 + k / 2] = h0 | (h1 << 16);
+              lw[2 * k4 + k / 2] = l0 | (l1 << 16);
+            }
+          }
+          tmem_st_16x32bx2_x8<72>(tmem + q_lanes + kColQ + 8u * (uint32_t)c, hw);
+          tmem_st_16x32bx2_x8<72>(tmem + q_lanes + kColQ + 144u + 8u * (uint32_t)c, lw);
+        }
+        tmem_wait_st();
+        if (lane < 16) s_qsc[h] = q_unscale;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(BAR_QT));
+      } else {
+        // the other warp of the quarter takes the head's scale once the
+        // query is in place
+        if (!mbar_wait(BAR(BAR_QT), 0, wl)) aborted = true;
+        q_unscale = s_qsc[h];
+      }
+    } else if (u == 0) {
+      // the query row into tensor memory: dims [kQK/2 half, +kQK/2), read
+      // from the copy staged in shared memory (row-major [64][kQK])
       bool okq = mbar_wait(BAR(BAR_QS), 0);
       if (okq) {
         const uint8_t* qrow = smem + kSmemKV + C::kQStage * kTileBytes + h * (kQK * 2) + half * kQK;
@@ -1089,9 +1349,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         for (int c = 0; c < kQK / 64; ++c) {
           uint32_t r[16];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qrow + c * 64 + u * 16);
-            r[4 * u] = v.x; r[4 * u + 1] = v.y; r[4 * u + 2] = v.z; r[4 * u + 3] = v.w;
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(qrow + c * 64 + k4 * 16);
+            r[4 * k4] = v.x; r[4 * k4 + 1] = v.y; r[4 * k4 + 2] = v.z; r[4 * k4 + 3] = v.w;
           }
           tmem_st_16x32bx2_x16<kQK / 4>(tmem + q_lanes + kColQ + 16u * (uint32_t)c, r);  // second half at +kQK/4
         }
@@ -1103,96 +1363,192 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     }
     // l_run: sum of the probabilities as fp32 (gives lse); l_pv: the same sum
     // of the bf16-rounded probabilities the PV MMA used (normalises out, so
-    // the output weights sum to one exactly).  fp8 rows fold the row scale
-    // into P, so there l_pv = l_run.
+    // the output weights sum to one exactly).
     float m_run = -INFINITY, l_run = 0.f, l_pv = 0.f;
-    bool aborted = false;
+    // fp8: O and its normaliser are kept times sig2 (0 until the first
+    // nonzero probability), the power of two of the e4m3 P parts
+    float sig2 = 0.f;
+    const float fsc = p.scale_log2 * q_unscale;
     for (int i = 0; i < ntiles; ++i) {
       const int sb = i & 1, rs = i % kRing;
-      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1, wl) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1, wl)) {
+      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1, wl) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1, wl))
         aborted = true;
+      aborted = __any_sync(0xffffffffu, aborted);
+      float s[kTok];
+      if (!aborted) {
+        tc_fence_after();
+        if constexpr (kTok == 32) tmem_ld_16x32bx2_x32(tmem + q_lanes + kColS + 64u * (uint32_t)sb, s);
+        else tmem_ld_16x32bx2_x16(tmem + q_lanes + kColS + 64u * (uint32_t)sb + (uint32_t)(kTok * u), s);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int j = 0; j < kTok; ++j) s[j] = 0.f;
       }
-      if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
-      tc_fence_after();
-      float s[32];
-      tmem_ld_16x32bx2_x32(tmem + q_lanes + kColS + 64u * (uint32_t)sb, s);
-      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_SE + sb));
 
-      int rows[32];
-      float rsc[32];
+      int rows[kTok];
+      float rsc[kTok];
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const int4 r4 = *reinterpret_cast<const int4*>(s_row + rs * 64 + half * 32 + j);
+      for (int j = 0; j < kTok; j += 4) {
+        const int4 r4 = *reinterpret_cast<const int4*>(s_row + rs * 64 + tok0 + j);
         rows[j] = r4.x; rows[j + 1] = r4.y; rows[j + 2] = r4.z; rows[j + 3] = r4.w;
         if (kFp8) {
-          const float4 c4 = *reinterpret_cast<const float4*>(s_rsc + rs * 64 + half * 32 + j);
+          const float4 c4 = *reinterpret_cast<const float4*>(s_rsc + rs * 64 + tok0 + j);
           rsc[j] = c4.x; rsc[j + 1] = c4.y; rsc[j + 2] = c4.z; rsc[j + 3] = c4.w;
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(BAR_IXE + rs));
-      float tmax = -INFINITY;
+      // logits in log2 units (padding: -inf) and this thread's maximum
+      float tm[kTok / 2];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float f = kFp8 ? p.scale_log2 * rsc[j] : p.scale_log2;
-        const float x = rows[j] >= 0 ? s[j] * f : -INFINITY;
-        s[j] = x;
-        tmax = fmaxf(tmax, x);
+      for (int j = 0; j < kTok; ++j) {
+        const float f = kFp8 ? fsc * rsc[j] : p.scale_log2;
+        s[j] = rows[j] >= 0 ? s[j] * f : -INFINITY;
       }
-      tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-      const float m_new = fmaxf(m_run, tmax);
-      const bool need = m_new > m_run + kRescaleThresh;
-      const float m_use = need ? m_new : m_run;
-      const float alpha = need ? ex2(m_run - m_use) : 1.f;
-      uint32_t pk[16];
-      float lsum = 0.f, lsum_pv = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float p0 = s[j] == -INFINITY ? 0.f : ex2(s[j] - m_use);
-        const float p1 = s[j + 1] == -INFINITY ? 0.f : ex2(s[j + 1] - m_use);
-        lsum += p0 + p1;
-        if constexpr (kFp8) {
-          pk[j / 2] = pack_bf16x2(p0 * rsc[j], p1 * rsc[j + 1]);
-        } else {
-          const uint32_t w = pack_bf16x2(p0, p1);
-          pk[j / 2] = w;
-          lsum_pv += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+      for (int j = 0; j < kTok / 2; ++j) tm[j] = fmaxf(s[2 * j], s[2 * j + 1]);
+#pragma unroll
+      for (int w2 = kTok / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int j = 0; j < w2; ++j) tm[j] = fmaxf(tm[j], tm[j + w2]);
+      // Probabilities against the running maximum, as long as no thread's
+      // logits pass it by more than the lazy threshold and (fp8) no thread's
+      // P' = p rsc leaves the range of the current power of two sig2.  One
+      // barrier of the softmax warps tells whether any thread needs an
+      // update (or gave up a wait); only then are the head's exact maxima
+      // exchanged and the probabilities recomputed.
+      float pr[kTok];
+      float lsum = 0.f, lsum_pv = 0.f;
+      uint32_t pk[kTok / 2];
+      auto probabilities = [&](float m_ref) -> float {   // returns this thread's largest |P'|
+        float pmx = 0.f;
+        lsum = 0.f;
+        lsum_pv = 0.f;
+#pragma unroll
+        for (int j = 0; j < kTok; j += 2) {
+          const float p0 = s[j] == -INFINITY ? 0.f : ex2(s[j] - m_ref);
+          const float p1 = s[j + 1] == -INFINITY ? 0.f : ex2(s[j + 1] - m_ref);
+          lsum += p0 + p1;
+          if constexpr (kNat) {
+            pr[j] = p0 * rsc[j];
+            pr[j + 1] = p1 * rsc[j + 1];
+            pmx = fmaxf(pmx, fmaxf(fabsf(pr[j]), fabsf(pr[j + 1])));
+          } else {
+            const uint32_t w = pack_bf16x2(p0, p1);
+            pk[j / 2] = w;
+            lsum_pv += __uint_as_float(w << 16) + __uint_as_float(w & 0xFFFF0000u);
+          }
+        }
+        return pmx;
+      };
+      // (every finite logit needs an update while m_run = -inf; the values
+      // computed against m_run are then discarded)
+      bool upd = tm[0] > m_run + kRescaleThresh;
+      float pmax = probabilities(upd ? tm[0] : m_run);
+      if constexpr (kNat) upd = upd || (pmax > 0.f && (sig2 == 0.f || pmax * sig2 >= 448.f));
+      float m_use = m_run, alpha = 1.f, r = 1.f;
+      bool need = false;
+      bool slow;
+      if constexpr (kU == 1) slow = __any_sync(0xffffffffu, upd || aborted);
+      else slow = group_any(upd || aborted, 2, 32 * kSmx);
+      if (slow) {
+        // the head's maximum over its 2 kU threads, then P against it
+        float tmax = fmaxf(tm[0], __shfl_xor_sync(0xffffffffu, tm[0], 16));
+        tmax = pair_reduce(tmax, true, aborted);
+        if (aborted) break;
+        const float m_new = fmaxf(m_run, tmax);
+        need = m_new > m_run + kRescaleThresh;
+        m_use = need ? m_new : m_run;
+        alpha = need ? ex2(m_run - m_use) : 1.f;
+        pmax = probabilities(m_use);
+        if constexpr (kNat) {
+          // P' goes to the MMA as e4m3 parts of P' sig2.  sig2 is set at the
+          // first tile with mass (its largest |P'| into [8, 16): values down
+          // to 2^-10 of it keep the parts' full 8 bits, and later tiles may
+          // grow 28-fold before anything changes) and lowered by a power of
+          // two r when a later tile's largest value would pass the e4m3
+          // maximum 448 (again into [8, 16)); O then takes the same factor.
+          pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 16));
+          pmax = pair_reduce(pmax, true, aborted);
+          if (pmax > 0.f) {
+            if (sig2 == 0.f) {
+              sig2 = pow2i(min(126, max(-126, 3 - ilog2f(pmax))));
+            } else {
+              const float tp = pmax * sig2;
+              if (tp >= 448.f) {
+                r = pow2i(max(-126, 3 - ilog2f(tp)));
+                sig2 *= r;
+              }
+            }
+          }
         }
       }
-      // Rescale this head's O row by alpha (O rows of the warp: lanes 16-31
-      // of its quarter; lane t and t+16 hold dims [0,256) and [256,512)).
-      // Only then must PV(i-1) have completed.  PVD[(i-1)&1] cannot be more
-      // than one phase behind: tile i was loaded after PV(i-3) released its
-      // stage, and PV(i+1) needs this warp's P(i+1).
-      const bool resc = need && i >= 1 && m_run > -INFINITY;
+      // Rescale this head's O row (this thread's chunks) by alpha r.  Only
+      // then must PV(i-1) have completed.  PVD[(i-1)&1] is at most one phase
+      // behind: PV(i-3) has completed (bf16 operands: tile i was loaded after
+      // PV(i-3) released its stage; fp8: this warp waited for PV(i-3) before
+      // writing P(i-1)), and PV(i+1) needs P(i+1).
+      const bool resc_m = need && i >= 1 && m_run > -INFINITY;
+      const bool resc = resc_m || r != 1.f;
       if (__any_sync(0xffffffffu, resc)) {
         if (!mbar_wait(BAR(BAR_PVD + ((i - 1) & 1)), ((i - 1) >> 1) & 1, wl)) aborted = true;
-        if (__any_sync(0xffffffffu, aborted)) { aborted = true; break; }
-        tc_fence_after();
-        const float f = resc ? alpha : 1.f;
+        aborted = __any_sync(0xffffffffu, aborted);
+        if (!aborted) {
+          tc_fence_after();
+          const float f = (resc_m ? alpha : 1.f) * r;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          float o[32];
-          const uint32_t ta = tmem + o_lanes + 32u * (uint32_t)c;
-          tmem_ld_16x32bx2_x32_h256(ta, o);
-          tmem_wait_ld();
+          for (int c = kOc * u; c < kOc * (u + 1); ++c) {
+            float o[32];
+            const uint32_t ta = tmem + o_lanes + 32u * (uint32_t)c;
+            tmem_ld_16x32bx2_x32_h256(ta, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= f;
-          tmem_st_16x32bx2_x32_h256(ta, o);
+            for (int k = 0; k < 32; ++k) o[k] *= f;
+            tmem_st_16x32bx2_x32_h256(ta, o);
+          }
+          tmem_wait_st();
         }
-        tmem_wait_st();
       }
       l_run = l_run * alpha + lsum;
-      l_pv = kFp8 ? l_run : l_pv * alpha + lsum_pv;
+      l_pv = l_pv * alpha + lsum_pv;
       m_run = m_use;
-      const uint32_t prow = sbase + kSmemKV + (i % kStages) * kTileBytes + kAtomP * kAtomBytes;
+      uint32_t prow;
+      if constexpr (kNat) {
+        // high and low e4m3 parts, four tokens per word
+        uint32_t hw[kTok / 4], lw[kTok / 4];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        st_shared_v4(prow + sw128_off(h, half * 4 + q4),
-                     make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]));
+        for (int j = 0; j < kTok; j += 4) {
+          uint32_t h0, l0, h1, l1;
+          split_e4m3x2_h(pr[j] * sig2, pr[j + 1] * sig2, h0, l0);
+          split_e4m3x2_h(pr[j + 2] * sig2, pr[j + 3] * sig2, h1, l1);
+          hw[j / 4] = h0 | (h1 << 16);
+          lw[j / 4] = l0 | (l1 << 16);
+        }
+        // P buffer i mod 2 is free once PV(i-2) has completed (which also
+        // keeps the PVD waits of tile i+1 at most one phase ahead)
+        if (i >= 2 && !mbar_wait(BAR(BAR_PVD + (i & 1)), ((i - 2) >> 1) & 1, wl)) aborted = true;
+        aborted = __any_sync(0xffffffffu, aborted);
+        if (aborted) continue;   // (the next exchange, or the epilogue's, stops every softmax warp)
+        // row h: codes [tok0, +kTok) high parts (16-token chunks tok0 / 16
+        // on), codes [64 + tok0, +kTok) low parts
+        prow = sbase + C::kSmemP + (uint32_t)((i & 1) * kAtomBytes);
+#pragma unroll
+        for (int k = 0; k < kTok / 16; ++k) {
+          st_shared_v4(prow + sw128_off(h, tok0 / 16 + k), make_uint4(hw[4 * k], hw[4 * k + 1], hw[4 * k + 2], hw[4 * k + 3]));
+          st_shared_v4(prow + sw128_off(h, 4 + tok0 / 16 + k),
+                       make_uint4(lw[4 * k], lw[4 * k + 1], lw[4 * k + 2], lw[4 * k + 3]));
+        }
+      } else {
+        if (aborted) continue;
+        // P(t) [64 heads][64 tokens] bf16 in the stage's rope atom: row h,
+        // 8-token chunks tok0 / 8 on
+        prow = sbase + kSmemKV + (i % kStages) * kTileBytes + kAtomP * kAtomBytes;
+#pragma unroll
+        for (int k = 0; k < kTok / 8; ++k)
+          st_shared_v4(prow + sw128_off(h, tok0 / 8 + k), make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]));
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -1207,37 +1563,44 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // PV(n-2) then PV(n-1): each wait is at most one phase ahead
       if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + (ntiles & 1)), ((ntiles - 2) >> 1) & 1, wl)) aborted = true;
       if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1, wl)) aborted = true;
-      aborted = __any_sync(0xffffffffu, aborted);
       tc_fence_after();
     }
+    // the head's totals over its kU warps (and the common abort decision)
+    float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+    l_tot = pair_reduce(l_tot, false, aborted);
+    // the normaliser of O (bf16 operands: the rounded-P sum; fp8: the
+    // probability sum times sig2) and the split's weight in a merge (the
+    // rounded-P sum; fp8: the probability sum)
+    float l_w = l_tot;
+    if constexpr (!kNat) {
+      l_w = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
+      l_w = pair_reduce(l_w, false, aborted);
+    }
+    const float l_nrm = kNat ? l_tot * sig2 : l_w;
     if (p.cluster) {
       // in-cluster merge (after the warp roles): this split's per-head
-      // statistics (max, fp32 sum, rounded-P sum) go to the workspace
+      // statistics (max, merge weight, fp32 sum) go to the workspace
       merge_failed = aborted;
-      const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
-      const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
-      if (!aborted && half == 0) {
+      if (!aborted && u == 0 && half == 0) {
         float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * kStatFloats;
-        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * kStatFloats) = make_float4(m_run, l_nrm, l_tot, 0.f);
-        // for the merge writers: 1 / (rounded-P sum) of head h
+        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * kStatFloats) = make_float4(m_run, l_w, l_tot, 0.f);
+        // for the merge writers: 1 / (normaliser of O) of head h
         reinterpret_cast<float*>(smem + C::kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
       }
     } else if (!aborted) {
-      const float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
-      const float l_nrm = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
       const bool any = l_tot > 0.f;
-      const float inv_l = any ? 1.f / l_nrm : 0.f;
+      const float inv_l = any && l_nrm > 0.f ? 1.f / l_nrm : 0.f;
       const float lse_h = any ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
       const bool direct = p.nsplit == 1;
       const size_t part = (size_t)b * p.nsplit + split;
-      // Stage this warp's 16 head rows in shared memory (the idle KV stages)
-      // with a 16-byte pad per row, which makes the 16-byte stores of a warp
+      // Stage the head rows in shared memory (the idle operand stages) with
+      // a 16-byte pad per row, which makes the 16-byte stores of a warp
       // conflict-free, then write each row with one bulk copy.
       const uint32_t row_bytes = direct ? kDv * 2 : kDv * 4;
       const uint32_t stride = row_bytes + 16;
       uint8_t* srow = smem + kSmemKV + (size_t)h * stride;
 #pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
+      for (int c = kOc * u; c < kOc * (u + 1); ++c) {
         float o[32];
         if (ntiles > 0) {
           tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
@@ -1250,28 +1613,28 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         if (direct) {
           uint4* dst = reinterpret_cast<uint4*>(srow + d0 * 2);
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            dst[u] = make_uint4(pack_bf16x2(o[8 * u] * inv_l, o[8 * u + 1] * inv_l),
-                                pack_bf16x2(o[8 * u + 2] * inv_l, o[8 * u + 3] * inv_l),
-                                pack_bf16x2(o[8 * u + 4] * inv_l, o[8 * u + 5] * inv_l),
-                                pack_bf16x2(o[8 * u + 6] * inv_l, o[8 * u + 7] * inv_l));
+          for (int k4 = 0; k4 < 4; ++k4)
+            dst[k4] = make_uint4(pack_bf16x2(o[8 * k4] * inv_l, o[8 * k4 + 1] * inv_l),
+                                 pack_bf16x2(o[8 * k4 + 2] * inv_l, o[8 * k4 + 3] * inv_l),
+                                 pack_bf16x2(o[8 * k4 + 4] * inv_l, o[8 * k4 + 5] * inv_l),
+                                 pack_bf16x2(o[8 * k4 + 6] * inv_l, o[8 * k4 + 7] * inv_l));
         } else {
           float4* dst = reinterpret_cast<float4*>(srow + d0 * 4);
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            dst[u] = make_float4(o[4 * u] * inv_l, o[4 * u + 1] * inv_l, o[4 * u + 2] * inv_l,
-                                 o[4 * u + 3] * inv_l);
+          for (int k4 = 0; k4 < 8; ++k4)
+            dst[k4] = make_float4(o[4 * k4] * inv_l, o[4 * k4 + 1] * inv_l, o[4 * k4 + 2] * inv_l,
+                                  o[4 * k4 + 3] * inv_l);
         }
       }
       fence_proxy_async_smem();
-      __syncwarp();
-      if (half == 0) {
+      // the row's other chunks come from the other warp of the quarter
+      if constexpr (kU == 2) named_bar_sync(2, 32 * kSmx);
+      else __syncwarp();
+      if (u == 0 && half == 0) {
         uint8_t* gdst = direct ? reinterpret_cast<uint8_t*>(p.out + ((size_t)b * kH + h) * kDv)
                                : reinterpret_cast<uint8_t*>(p.part_o + (part * kH + h) * kDv);
         bulk_store_s2g(gdst, smem_u32(srow), row_bytes);
         bulk_commit();
-      }
-      if (half == 0) {
         if (direct) p.lse[(size_t)b * kH + h] = lse_h;
         else p.part_lse[part * kH + h] = lse_h;
         bulk_wait_all();
