@@ -84,7 +84,7 @@ constexpr int kRawTileBytes = kTile * kRawRowBytes; // 36,864
 // contiguous bytes per row, before conversion to bf16.
 // fp8 caches compute on the codes as stored: an operand stage is one tile
 // of 576-code rows as 8-row x 16-byte core matrices (no swizzle; K-major
-// for S, MN-major for PV), and P(t) goes to one of two separate P buffers
+// for S, MN-major for PV), and P(t) goes to one of four separate P buffers
 // ([64 heads][128 codes: 64 tokens high part, 64 low part], 128-byte
 // swizzled, K-major).
 constexpr int kSmemKV = 0;
@@ -97,8 +97,8 @@ constexpr int BAR_KVE = BAR_KVF + kMaxStages;       // [stages] operand tile con
 constexpr int BAR_SF = BAR_KVE + kMaxStages;        // [2] S(t) in TMEM
 constexpr int BAR_SE = BAR_SF + 2;                  // [2] S(t) read by the softmax
 constexpr int BAR_PF = BAR_SE + 2;                  // [stages] P(t) written (per stage)
-constexpr int BAR_PVD = BAR_PF + kMaxStages;        // [2] PV(t) done (by tile parity)
-constexpr int BAR_FIN = BAR_PVD + 2;                // drain, S issuer
+constexpr int BAR_PVD = BAR_PF + kMaxStages;        // [4] PV(t) done (by t mod 4)
+constexpr int BAR_FIN = BAR_PVD + 4;                // drain, S issuer
 constexpr int BAR_FIN2 = BAR_FIN + 1;               // drain, PV issuer
 constexpr int BAR_QT = BAR_FIN2 + 1;                // query written to TMEM
 constexpr int BAR_QS = BAR_QT + 1;                  // query staged in shared memory
@@ -182,8 +182,8 @@ struct Cfg {
   static constexpr int kCpGroups = kConv ? 5 : 8;
   static constexpr int kBulkGroups = 8 - kCpGroups;      // one expect-tx arrival each
   // shared memory map
-  static constexpr int kSmemP = kSmemKV + kStages * kOpBytes;             // fp8: two P buffers
-  static constexpr int kSmemRaw = kSmemP + (kNat ? 2 * kAtomBytes : 0);
+  static constexpr int kSmemP = kSmemKV + kStages * kOpBytes;             // fp8: four P buffers
+  static constexpr int kSmemRaw = kSmemP + (kNat ? 4 * kAtomBytes : 0);
   static constexpr int kSmemAux = kSmemRaw + kRawStages * kRawTileBytes;
   static constexpr int kAuxBars = kSmemAux;
   static constexpr int kAuxTmem = (kAuxBars + 8 * kNumBars + 15) / 16 * 16;  // TMEM base address (4 B)
@@ -838,8 +838,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(BAR_SF + s), 1);
       mbar_init(BAR(BAR_SE + s), kSmx);
-      mbar_init(BAR(BAR_PVD + s), 1);
     }
+    for (int s = 0; s < 4; ++s) mbar_init(BAR(BAR_PVD + s), 1);
     mbar_init(BAR(BAR_FIN), 1);
     mbar_init(BAR(BAR_FIN2), 1);
     mbar_init(BAR(BAR_QT), 4);
@@ -1207,12 +1207,12 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         tc_fence_after();
         if constexpr (kNat) {
           // O[:, 256 hf + n] += P8[:, 32 kk + k] V[32 (kk mod 2) + k, 256 hf + n]:
-          // A = P buffer t mod 2 (codes 0-63: high parts of the 64 tokens,
+          // A = P buffer t mod 4 (codes 0-63: high parts of the 64 tokens,
           // 64-127: low parts; K step +32 B), B = the stage's codes
           // MN-major (8-token groups 4608 B apart, 16-dim chunks 128 B
           // apart; dims 256 hf = chunk 16 hf)
           const uint32_t vb = sbase + kSmemKV + stage * C::kOpBytes;
-          const uint64_t dp = sw128_desc(sbase + C::kSmemP + (t & 1) * kAtomBytes, 16, 1024);
+          const uint64_t dp = sw128_desc(sbase + C::kSmemP + (t & 3) * kAtomBytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
@@ -1242,7 +1242,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
           }
         }
         commit_elect(BAR(BAR_KVE + stage));
-        commit_elect(BAR(BAR_PVD + (t & 1)));
+        commit_elect(BAR(BAR_PVD + (t & 3)));
       }
     }
     // drain: every MMA this warp issued has completed before teardown
@@ -1256,8 +1256,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // lane / 16, u = w / 4); of O it holds dims [256 half, +256), 32-dim
     // chunks [kOc u, kOc u + kOc).  With two warps per quarter a head's
     // maxima and sums are combined through shared memory at a barrier of
-    // the softmax warps, which also ORs their abort flags: every softmax
-    // warp leaves the tile loop at the same tile.
+    // the quarter's two warps (named barrier 2 + q), which also ORs their
+    // abort flags: both leave the tile loop at the same tile.
     constexpr int kU = kSmx / 4, kTok = 32 / kU, kOc = 8 / kU;
     const int q = warp & 3, u = warp >> 2;
     const int h = 16 * q + (lane & 15);
@@ -1277,7 +1277,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         float* x = s_xch + (xc & 1) * (2 * 64);
         ++xc;
         if (lane < 16) x[u * 64 + h] = v;
-        ab = group_any(ab, 2, 32 * kSmx);
+        ab = group_any(ab, 2 + q, 64);
         const float o = x[(1 - u) * 64 + h];
         return is_max ? fmaxf(v, o) : v + o;
       }
@@ -1417,9 +1417,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // Probabilities against the running maximum, as long as no thread's
       // logits pass it by more than the lazy threshold and (fp8) no thread's
       // P' = p rsc leaves the range of the current power of two sig2.  One
-      // barrier of the softmax warps tells whether any thread needs an
-      // update (or gave up a wait); only then are the head's exact maxima
-      // exchanged and the probabilities recomputed.
+      // barrier of the quarter's warps tells whether any of their threads
+      // needs an update (or gave up a wait); only then are the heads' exact
+      // maxima exchanged and the probabilities recomputed.
       float pr[kTok];
       float lsum = 0.f, lsum_pv = 0.f;
       uint32_t pk[kTok / 2];
@@ -1453,7 +1453,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       bool need = false;
       bool slow;
       if constexpr (kU == 1) slow = __any_sync(0xffffffffu, upd || aborted);
-      else slow = group_any(upd || aborted, 2, 32 * kSmx);
+      else slow = group_any(upd || aborted, 2 + q, 64);
       if (slow) {
         // the head's maximum over its 2 kU threads, then P against it
         float tmax = fmaxf(tm[0], __shfl_xor_sync(0xffffffffu, tm[0], 16));
@@ -1487,14 +1487,14 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         }
       }
       // Rescale this head's O row (this thread's chunks) by alpha r.  Only
-      // then must PV(i-1) have completed.  PVD[(i-1)&1] is at most one phase
-      // behind: PV(i-3) has completed (bf16 operands: tile i was loaded after
-      // PV(i-3) released its stage; fp8: this warp waited for PV(i-3) before
-      // writing P(i-1)), and PV(i+1) needs P(i+1).
+      // then must PV(i-1) have completed.  PVD[(i-1) mod 4] is at most one
+      // phase behind: PV(i-5) has completed (bf16 operands: tile i was
+      // loaded after PV(i-3) released its stage; fp8: this warp waited for
+      // PV(i-5) before writing P(i-1)), and PV(i+3) needs P(i+3).
       const bool resc_m = need && i >= 1 && m_run > -INFINITY;
       const bool resc = resc_m || r != 1.f;
       if (__any_sync(0xffffffffu, resc)) {
-        if (!mbar_wait(BAR(BAR_PVD + ((i - 1) & 1)), ((i - 1) >> 1) & 1, wl)) aborted = true;
+        if (!mbar_wait(BAR(BAR_PVD + ((i - 1) & 3)), ((i - 1) >> 2) & 1, wl)) aborted = true;
         aborted = __any_sync(0xffffffffu, aborted);
         if (!aborted) {
           tc_fence_after();
@@ -1527,14 +1527,14 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
           hw[j / 4] = h0 | (h1 << 16);
           lw[j / 4] = l0 | (l1 << 16);
         }
-        // P buffer i mod 2 is free once PV(i-2) has completed (which also
+        // P buffer i mod 4 is free once PV(i-4) has completed (which also
         // keeps the PVD waits of tile i+1 at most one phase ahead)
-        if (i >= 2 && !mbar_wait(BAR(BAR_PVD + (i & 1)), ((i - 2) >> 1) & 1, wl)) aborted = true;
+        if (i >= 4 && !mbar_wait(BAR(BAR_PVD + (i & 3)), ((i - 4) >> 2) & 1, wl)) aborted = true;
         aborted = __any_sync(0xffffffffu, aborted);
         if (aborted) continue;   // (the next exchange, or the epilogue's, stops every softmax warp)
         // row h: codes [tok0, +kTok) high parts (16-token chunks tok0 / 16
         // on), codes [64 + tok0, +kTok) low parts
-        prow = sbase + C::kSmemP + (uint32_t)((i & 1) * kAtomBytes);
+        prow = sbase + C::kSmemP + (uint32_t)((i & 3) * kAtomBytes);
 #pragma unroll
         for (int k = 0; k < kTok / 16; ++k) {
           st_shared_v4(prow + sw128_off(h, tok0 / 16 + k), make_uint4(hw[4 * k], hw[4 * k + 1], hw[4 * k + 2], hw[4 * k + 3]));
@@ -1561,8 +1561,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     if (threadIdx.x == 0) grid_dep_launch();
     if (!aborted && ntiles > 0) {
       // PV(n-2) then PV(n-1): each wait is at most one phase ahead
-      if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + (ntiles & 1)), ((ntiles - 2) >> 1) & 1, wl)) aborted = true;
-      if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 1)), ((ntiles - 1) >> 1) & 1, wl)) aborted = true;
+      if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + ((ntiles - 2) & 3)), ((ntiles - 2) >> 2) & 1, wl)) aborted = true;
+      if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 3)), ((ntiles - 1) >> 2) & 1, wl)) aborted = true;
       tc_fence_after();
     }
     // the head's totals over its kU warps (and the common abort decision)
@@ -1628,7 +1628,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       }
       fence_proxy_async_smem();
       // the row's other chunks come from the other warp of the quarter
-      if constexpr (kU == 2) named_bar_sync(2, 32 * kSmx);
+      if constexpr (kU == 2) named_bar_sync(2 + q, 64);
       else __syncwarp();
       if (u == 0 && half == 0) {
         uint8_t* gdst = direct ? reinterpret_cast<uint8_t*>(p.out + ((size_t)b * kH + h) * kDv)
