@@ -1066,18 +1066,27 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1, wl)))
           break;
         // fp8 rows as stored, into the core-matrix layout: chunk c (0..35)
-        // of a row to cm_off(row in tile, c)
+        // of a row to cm_off(row in tile, c).  One instruction per row for
+        // its first 512 bytes (lane = chunk), then one for the last 64 bytes
+        // of the group's eight rows (lane = 4 row + chunk - 32): per 128-byte
+        // line of a gathered row this issues fewer requests than eight rows x
+        // 64 bytes per instruction, which measured ~7 % faster on 576-byte
+        // rows although each 512-byte instruction meets bank conflicts on
+        // the shared-memory side.
         const uint32_t tbase = sbase + kSmemKV + stage * C::kOpBytes;
 #pragma unroll
         for (int gi = 0; gi < kGpw; ++gi) {
-          const int tok = 8 * (lw + C::kCopyWarps * gi) + r8;
-          const int row = rows[gi];
-          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8;
-          const uint32_t nbytes = row >= 0 ? 16u : 0u;
+          const int g = lw + C::kCopyWarps * gi;
 #pragma unroll
-          for (int sg = 0; sg < 9; ++sg) {
-            const int c = 4 * sg + c4;
-            cp_async_16(tbase + cm_off(tok, c), src + c * 16, nbytes);
+          for (int rr = 0; rr < 8; ++rr) {
+            const int row = __shfl_sync(0xffffffffu, rows[gi], 4 * rr);   // lane 4 rr holds row 8 g + rr
+            const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8;
+            cp_async_16(tbase + cm_off(8 * g + rr, lane), src + lane * 16, row >= 0 ? 16u : 0u);
+          }
+          {
+            const int row = rows[gi];                                     // row 8 g + r8
+            const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesFp8;
+            cp_async_16(tbase + cm_off(8 * g + r8, 32 + c4), src + (32 + c4) * 16, row >= 0 ? 16u : 0u);
           }
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
