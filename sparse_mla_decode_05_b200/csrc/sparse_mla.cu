@@ -1096,18 +1096,28 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         // the last stage first holds the staged query
         if (__any_sync(0xffffffffu, t == C::kQStage && !mbar_wait(BAR(BAR_QT), 0, wl))) break;
         // bf16 rows straight into the swizzled operand tile: chunk c (0..71)
-        // of a row is 16-byte chunk c % 8 of atom c / 8
+        // of a row is 16-byte chunk c % 8 of atom c / 8.  Two instructions
+        // per row for its first 1,024 bytes (lane = chunk), then two for the
+        // last 128 bytes of the group's eight rows (lane = 8 row + chunk - 64
+        // over four rows each).
         const uint32_t tbase = sbase + kSmemKV + stage * kTileBytes;
+        auto copy_chunk = [&](int tok, int row, int c) {
+          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16;
+          cp_async_16(tbase + (c >> 3) * kAtomBytes + sw128_off(tok, c & 7), src + c * 16, row >= 0 ? 16u : 0u);
+        };
 #pragma unroll
         for (int gi = 0; gi < kGpw; ++gi) {
-          const int tok = 8 * (lw + C::kCopyWarps * gi) + r8;
-          const int row = rows[gi];
-          const uint8_t* src = p.kv + (size_t)(row >= 0 ? row : 0) * kRowBytesBf16;
-          const uint32_t nbytes = row >= 0 ? 16u : 0u;
+          const int g = lw + C::kCopyWarps * gi;
 #pragma unroll
-          for (int sg = 0; sg < 18; ++sg) {
-            const int c = 4 * sg + c4;
-            cp_async_16(tbase + (c >> 3) * kAtomBytes + sw128_off(tok, c & 7), src + c * 16, nbytes);
+          for (int rr = 0; rr < 8; ++rr) {
+            const int row = __shfl_sync(0xffffffffu, rows[gi], 4 * rr);   // lane 4 rr holds row 8 g + rr
+            copy_chunk(8 * g + rr, row, lane);
+            copy_chunk(8 * g + rr, row, 32 + lane);
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int rr = 4 * hh + (lane >> 3);
+            copy_chunk(8 * g + rr, __shfl_sync(0xffffffffu, rows[gi], 4 * rr), 64 + (lane & 7));
           }
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_KVF + stage));
@@ -1134,15 +1144,17 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
             __syncwarp();
             if (v) bulk_load_g2s(rbase + (8 * g + lane) * kRawRowBytes, row_src(brow[gi]), kRawRowBytes, BAR(BAR_RAW + rst));
           } else {
-            const int tok = 8 * g + r8;
-            const int row = rows[gi];
-            const uint8_t* src = row_src(row >= 0 ? row : 0);
-            const uint32_t nbytes = row >= 0 ? 16u : 0u;
+            // one instruction per row for its first 512 bytes (lane =
+            // chunk), one for the last 64 bytes of the group's eight rows
 #pragma unroll
-            for (int sg = 0; sg < 9; ++sg) {
-              const int c = 4 * sg + c4;
-              cp_async_16(rbase + tok * kRawRowBytes + c * 16, src + c * 16, nbytes);
+            for (int rr = 0; rr < 8; ++rr) {
+              const int row = __shfl_sync(0xffffffffu, rows[gi], 4 * rr);   // lane 4 rr holds row 8 g + rr
+              cp_async_16(rbase + (8 * g + rr) * kRawRowBytes + lane * 16, row_src(row >= 0 ? row : 0) + lane * 16,
+                          row >= 0 ? 16u : 0u);
             }
+            const int row = rows[gi];                                       // row 8 g + r8
+            cp_async_16(rbase + (8 * g + r8) * kRawRowBytes + (32 + c4) * 16, row_src(row >= 0 ? row : 0) + (32 + c4) * 16,
+                        row >= 0 ? 16u : 0u);
           }
         }
         cp_async_mbar_arrive_noinc(BAR(BAR_RAW + rst));
