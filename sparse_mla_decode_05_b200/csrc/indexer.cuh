@@ -31,9 +31,10 @@ constexpr int kIxAtomK = kIxTile * 128;          // one 64-dim half of K: 128 ro
 constexpr int kIxSmemQ = 0;
 constexpr int kIxSmemK = kIxSmemQ + kIxQBytes;
 constexpr int kIxSmemW = kIxSmemK + kIxKBytes;   // w [64] fp32
-constexpr int kIxSmemBar = kIxSmemW + kIxH * 4;  // mbarrier (8 B)
-constexpr int kIxSmemTmem = kIxSmemBar + 8;      // tensor-memory base address (4 B)
-constexpr int kIxSmemBytes = kIxSmemTmem + 8;    // 49,424: four CTAs per SM
+constexpr int kIxSmemBar = kIxSmemW + kIxH * 4;  // mbarrier: the MMA (8 B)
+constexpr int kIxSmemBarK = kIxSmemBar + 8;      // mbarrier: the key copies (8 B)
+constexpr int kIxSmemTmem = kIxSmemBarK + 8;     // tensor-memory base address (4 B)
+constexpr int kIxSmemBytes = kIxSmemTmem + 8;    // 49,432: four CTAs per SM
 constexpr uint32_t kIxTmemCols = 64;             // D: 128 lanes (positions) x 64 columns (heads)
 constexpr uint32_t kIdescIx = make_idesc(128, 64, false, false);
 static_assert(kIxSmemK % 1024 == 0 && kIxAtomQ % 1024 == 0 && kIxAtomK % 1024 == 0,
@@ -45,7 +46,10 @@ constexpr int kTkThreads = 1024;                 // top-k: one CTA per sequence
 static_assert(sizeof(smla_indexer_shape) == 40 && offsetof(smla_indexer_shape, num_key_rows) == 32,
               "smla_indexer_shape layout");
 
-struct IndexerParams {
+struct alignas(64) IndexerParams {
+  // the key cache as a 2-D tensor map: [num_rows][128] bf16, box 64 dims x
+  // 64 rows, 128-byte swizzle (one half of a page lands as one operand atom)
+  CUtensorMap kmap;
   const uint8_t* q;            // [B, 64, 128] bf16
   const float* w;              // [B, 64]
   const uint8_t* k;            // [num_rows, 128] bf16
@@ -74,8 +78,10 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32
 }
 
 // One CTA per (tile of 128 positions, sequence).  The tile's keys (two
-// pages, each 64 contiguous rows of 256 B) and the sequence's query are
-// staged 128B-swizzled, K-major; one elected thread issues
+// pages, each 64 contiguous rows of 256 B) come by tensor copies (four, one
+// per page and 64-dim half, 128-byte swizzle applied by the copy engine),
+// the sequence's query by 16-byte cp.async, both K-major; one elected
+// thread issues
 // D[128 x 64] = K . Q^T (eight K steps of 16) into tensor memory; then
 // thread t of warp w takes position 32 w + t: its 64 head dot products,
 // ReLU, weighted by w and summed in fp32, head by head.  Positions past the
@@ -98,9 +104,10 @@ __global__ void __launch_bounds__(kIxThreads) smla_indexer_score_kernel(const __
     if (s0 + t < p.max_ctx) srow[s0 + t] = -INFINITY;
     return;
   }
-  const uint32_t bar = sbase + kIxSmemBar;
+  const uint32_t bar = sbase + kIxSmemBar, bark = sbase + kIxSmemBarK;
   if (t == 0) {
     mbar_init(bar, 1);
+    mbar_init(bark, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -117,8 +124,9 @@ __global__ void __launch_bounds__(kIxThreads) smla_indexer_score_kernel(const __
     cp_async_16(sbase + kIxSmemQ + (j >> 3) * kIxAtomQ + sw128_off(row, j & 7), qb + (size_t)c * 16, 16u);
   }
   // the keys: positions s0 .. s0 + 127 lie in pages s0 / 64 and s0 / 64 + 1
-  // of the sequence (the host keeps max_ctx <= 64 pages_per_seq); 16 lanes
-  // per 256-byte row, so each warp instruction reads two whole rows
+  // of the sequence (the host keeps max_ctx <= 64 pages_per_seq).  A page
+  // at or past the context, or outside the cache, is zero-filled instead
+  // (its positions score -inf, or 0 when within the context: read as absent).
   long long rbase[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -129,14 +137,25 @@ __global__ void __launch_bounds__(kIxThreads) smla_indexer_score_kernel(const __
       else if (t == 0) atomicOr(&g_error_word, 4u);   // page outside the cache: read as absent
     }
   }
+  if (t == 0) {
+    const uint32_t nk = (rbase[0] >= 0 ? 2u : 0u) + (rbase[1] >= 0 ? 2u : 0u);
+    mbar_arrive_expect_tx(bark, nk * 64u * 128u);
 #pragma unroll
-  for (int u = 0; u < kIxKBytes / 16 / kIxThreads; ++u) {
-    const int c = u * kIxThreads + t;
-    const int r = c >> 4, j = c & 15;
-    const long long rb = rbase[r >> 6];
-    const bool ok = s0 + r < ctx && rb >= 0;
-    const uint8_t* src = ok ? p.k + (size_t)(rb + (r & 63)) * (kIxD * 2) + (size_t)j * 16 : p.k;
-    cp_async_16(sbase + kIxSmemK + (j >> 3) * kIxAtomK + sw128_off(r, j & 7), src, ok ? 16u : 0u);
+    for (int h = 0; h < 2; ++h) {
+      if (rbase[h] < 0) continue;
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+        tma_load_2d(sbase + kIxSmemK + half * kIxAtomK + h * 64 * 128, &p.kmap, 64 * half, (int)rbase[h], bark);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (rbase[h] >= 0) continue;
+#pragma unroll
+    for (int u = 0; u < 2 * 64 * 128 / 16 / kIxThreads; ++u) {
+      const int c = u * kIxThreads + t;                 // 16-byte unit of the page's two halves
+      st_shared_v4(sbase + kIxSmemK + (c >> 9) * kIxAtomK + h * 64 * 128 + (c & 511) * 16, make_uint4(0u, 0u, 0u, 0u));
+    }
   }
   float* ws = reinterpret_cast<float*>(smem + kIxSmemW);
   if (t < kIxH) ws[t] = __ldg(p.w + (size_t)b * kIxH + t);
@@ -146,7 +165,10 @@ __global__ void __launch_bounds__(kIxThreads) smla_indexer_score_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kIxSmemTmem);
-  if (warp == 0) {
+  // the key copies have landed (every thread waits: the copy engine's writes
+  // are then visible to the MMA issued below)
+  const bool keys_ok = mbar_wait(bark, 0);
+  if (warp == 0 && keys_ok) {
     const uint64_t da = sw128_desc(sbase + kIxSmemK, 16, 1024);
     const uint64_t db = sw128_desc(sbase + kIxSmemQ, 16, 1024);
 #pragma unroll
@@ -159,7 +181,7 @@ __global__ void __launch_bounds__(kIxThreads) smla_indexer_score_kernel(const __
     }
     commit_elect(bar);
   }
-  const bool ok = mbar_wait(bar, 0);
+  const bool ok = keys_ok && mbar_wait(bar, 0);
   tc_fence_after();
   float acc = 0.f;
   if (ok) {
@@ -499,6 +521,21 @@ static cudaError_t launch_pdl(const void* kern, dim3 grid, dim3 block, size_t sm
   return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (looked
+// up once; null if the driver does not offer it)
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult qr = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
 static smla_status run_indexer_scores(const smla_indexer_shape* s, const void* q, const float* w, const void* k,
                                       const int32_t* page_table, const int32_t* ctx_len, float* scores,
                                       cudaStream_t stream) {
@@ -512,6 +549,17 @@ static smla_status run_indexer_scores(const smla_indexer_shape* s, const void* q
     attr_done[dev] = 1;
   }
   IndexerParams prm;
+  // the key cache as a tensor map (host-side encoding, no device call)
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return SMLA_ERR_CUDA;
+  const cuuint64_t dims[2] = {(cuuint64_t)kIxD, (cuuint64_t)s->num_key_rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kIxD * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&prm.kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(k), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return SMLA_ERR_CUDA;
   prm.q = static_cast<const uint8_t*>(q);
   prm.w = w;
   prm.k = static_cast<const uint8_t*>(k);
