@@ -213,7 +213,7 @@ class Batches:
         self.plans = [api.DecodePlan(x.q.to(dev), self.kv, x.indices.to(dev), w.scale, kv_row_scale=self.rsc,
                                      page_table=self.pt, page_size=w.page_size) for x in self.ws]
         p0 = self.plans[0]
-        self.nsplit, self.clustered = p0.nsplit, p0.clustered
+        self.nsplit, self.clustered, self.streamk = p0.nsplit, p0.clustered, p0.streamk
         self.launches_per_step = 1 + (1 if p0.nsplit > 1 and not p0.clustered else 0)
         self.alg_bytes = float(np.mean([inputs.algorithmic_bytes(x) for x in self.ws]))
         self.alg_flops = float(np.mean([inputs.algorithmic_flops(x) for x in self.ws]))
@@ -424,7 +424,9 @@ def main():
             "traffic": kernel_traffic(args.workload), "algorithmic_bytes": bt.alg_bytes,
             "kernel": "smla_split_kernel", "peak_source": f"{peak_src} (copy)",
             "split_kernel_us": sp_ms * 1e3, "nsplit": bt.nsplit,
-            "split_reduction": "cluster (on chip)" if bt.clustered else ("partials + combine" if bt.nsplit > 1 else "none"),
+            "split_reduction": ("stream-K (rows shared by up to 3 CTAs, merged by the last)" if bt.streamk else
+                                "cluster (on chip)" if bt.clustered else
+                                ("partials + combine" if bt.nsplit > 1 else "none")),
             "roofline_us": rl_us, "frac_of_step_roofline": rl_us / (ms * 1e3),
             "frac_vs_nominal_8TBps": achieved / 8000.0,
             "note": "achieved = algorithmic bytes per launch / mean launch time over the timed region"}
@@ -515,6 +517,7 @@ def main():
             rl = roofline_us(ab, fl, peak_gbs, peak_tf)
             per_config.append({"workload": name, "batch": bc.w.batch, "tokens_per_seq": bc.w.tokens,
                                "topk": bc.w.topk, "nsplit": bc.nsplit, "clustered": bc.clustered,
+                               "streamk": bc.streamk,
                                "us_per_step": mc * 1e3, "gbs": ab / (mc * 1e-3) / 1e9, "roofline_us": rl,
                                "frac_roofline": rl / (mc * 1e3), "timing": note,
                                "cold_call_us": med, "cold_p10_us": p10, "cold_p90_us": p90,

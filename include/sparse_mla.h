@@ -120,10 +120,15 @@ typedef struct {
   int32_t pages_per_seq;  /* width of page_table when page_size > 0           */
   int32_t nsplit;         /* 0: the planner picks the top-k split; >= 1
                              forces that many splits (clamped to the number
-                             of 64-entry tiles of the list)                    */
+                             of 64-entry tiles of the list);
+                             SMLA_NSPLIT_STREAMK asks for the stream-K plan
+                             (see sparse_mla_plan_nsplit)                      */
   int32_t tokens_per_seq; /* T: query tokens per sequence, 0 or 1 = one token,
                              at most 16                                        */
 } smla_shape;
+
+/* smla_shape.nsplit value that asks for the stream-K plan. */
+#define SMLA_NSPLIT_STREAMK (-1)
 
 /* ABI version of the loaded library (SMLA_ABI_VERSION). */
 int32_t sparse_mla_abi_version(void);
@@ -148,18 +153,44 @@ const char* sparse_mla_status_string(smla_status status);
  * kernel.  Otherwise each split writes an fp32
  * partial result and a second (combine) kernel merges them.  An automatic
  * plan (shape->nsplit == 0) takes the largest such power of two for which
- * all clusters are resident at once. */
+ * all clusters are resident at once.
+ *
+ * Stream-K (shape->nsplit == SMLA_NSPLIT_STREAMK; this call then returns
+ * 1): for fp8 rows (SMLA_KV_FP8_E4M3_ROWSCALE) with lists of at least 16
+ * tiles of 64 entries, when there are more decode rows than half the SMs
+ * but not a whole multiple of them, one split per row leaves SMs idle or
+ * runs a short second wave.  Instead the grid has one CTA per SM, the rows'
+ * tiles are laid end to end (row-major) and each CTA takes an equal run of
+ * them.  A row then falls to one CTA, written out directly, or to two or
+ * three (consecutive) CTAs: each writes its part, normalised by its own
+ * softmax sum, with its log-sum-exp, to the workspace and counts itself in
+ * at the row's counter; the last to arrive merges the parts with the
+ * log-sum-exp combine ([Truth] "The Split-K Solution"), summing them in
+ * CTA order so that the bits do not depend on which CTA merges.  No CTA
+ * waits for another.  One kernel launch.  Other shapes that ask for it get
+ * the automatic plan.  (On B200 each CTA's switch to its second row costs
+ * more than the balance gains on the lists measured, so the automatic
+ * plan does not choose it.) */
 int32_t sparse_mla_plan_nsplit(const smla_shape* shape);
 
 /* How sparse_mla_decode merges the splits of `shape` on the current device:
  * 0 = one split (nothing to merge), 1 = inside the split kernel (thread-block
- * cluster, one launch), 2 = partials and the combine kernel (two launches).
- * Returns -1 if `shape` is invalid. */
+ * cluster, one launch), 2 = partials and the combine kernel (two launches),
+ * 3 = stream-K (one CTA per SM over the rows' tiles, a shared row merged
+ * by its last CTA; one launch).  Returns -1 if `shape` is invalid. */
 int32_t sparse_mla_plan_merge(const smla_shape* shape);
 
 /* Bytes of device workspace sparse_mla_decode needs for `shape` (0 when the
- * plan uses one split).  Deterministic in the shape, so a workspace sized
- * once per batch bucket can be reused by every call and every graph replay.
+ * plan uses one split).  Deterministic in the shape and the device's SM
+ * count, so a workspace sized once per batch bucket can be reused by every
+ * call and every graph replay.  A stream-K plan over G SMs needs
+ * 2 G x 64 x 512 fp32 part results, 2 G x 64 fp32 log-sum-exps and one
+ * 8-byte counter per (decode row, lane quarter of 16 heads), each region
+ * rounded up to 256 bytes (about 38 MB on 148 SMs).  The counters are
+ * tagged per launch and left at zero by the CTA that merges the row, so
+ * they need no initialisation either; after a call that set the device
+ * error word (a bounded wait gave up), replaying a graph captured before
+ * it on the same workspace is not supported.
  * Returns 0 for an invalid shape. */
 size_t sparse_mla_workspace_size(const smla_shape* shape);
 
@@ -192,7 +223,7 @@ smla_status sparse_mla_decode(const smla_shape* shape, const void* q, const void
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* The split kernel alone, always in its partials form (never the on-chip
- * merge), with the split count sparse_mla_plan_nsplit gives.
+ * merge, never stream-K), with the split count sparse_mla_plan_nsplit gives.
  * With nsplit == 1 it writes out/lse directly (workspace unused).  With
  * nsplit > 1 it writes per-split partial results into the workspace, which
  * must hold B*nsplit*64*(512+1)*4 bytes rounded up to a multiple of 256:

@@ -16,6 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsparse_mla.so")
 
 H, D_QK, D_V, TILE = 64, 576, 512, 64
+NSPLIT_STREAMK = -1          # smla_shape.nsplit asking for the stream-K plan
 KV_BF16, KV_FP8_E4M3_ROWSCALE, KV_DSV4_PAGED = 0, 1, 2
 DSV4_PAGE_BYTES, DSV4_D_QK = 37376, 512   # DeepSeek-V4 page: 64 x 576 slot bytes + 64 x 8 scale bytes
 
@@ -142,7 +143,8 @@ def plan_nsplit(shape: SmlaShape) -> int:
 
 def plan_merge(shape: SmlaShape) -> int:
     """0: one split; 1: splits merged inside the split kernel (cluster);
-    2: partials merged by the combine kernel."""
+    2: partials merged by the combine kernel; 3: stream-K (one CTA per SM
+    over the rows' tiles, a shared row merged by its last CTA)."""
     return lib.sparse_mla_plan_merge(ctypes.byref(shape))
 
 
@@ -323,8 +325,11 @@ class DecodePlan:
         self.shape = shape_for(q, kv, indices, page_table=page_table, page_size=page_size, nsplit=nsplit)
         dev = q.device
         self.nsplit = plan_nsplit(self.shape)
-        # the splits merge inside the split kernel (one launch, no combine)
-        self.clustered = plan_merge(self.shape) == 1
+        self.merge = plan_merge(self.shape)
+        # the splits merge inside the split kernel (one launch, no combine):
+        # in a thread-block cluster, or (stream-K) by the last CTA of a row
+        self.clustered = self.merge == 1
+        self.streamk = self.merge == 3
         o_shape, l_shape = _result_shapes(q)
         self.out = out if out is not None else torch.empty(o_shape, dtype=torch.bfloat16, device=dev)
         self.lse = lse if lse is not None else torch.empty(l_shape, dtype=torch.float32, device=dev)
@@ -353,7 +358,7 @@ class DecodePlan:
 
     def run_split(self, stream=None):
         """The split kernel of run(): all of run() when the splits reduce on chip."""
-        if self.clustered:
+        if self.clustered or self.streamk:
             return self.run(stream)
         st = lib.sparse_mla_decode_split(*self._split_args, self._stream if stream is None else stream)
         if st != 0:

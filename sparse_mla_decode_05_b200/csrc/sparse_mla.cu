@@ -54,6 +54,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "sparse_mla.h"
@@ -93,12 +94,14 @@ constexpr int kSmemKV = 0;
 constexpr int kAtomP = kAtoms - 1;
 constexpr int kRing = 4;                            // resolved-row ring depth (tiles)
 constexpr int kMaxStages = 5;
+constexpr int kNumS = 3;                            // S buffers in tensor memory
+constexpr int kMaxPieces = 3;                       // stream-K: CTAs that may share one row (rows > G / 2)
 // barrier indices
 constexpr int BAR_KVF = 0;                          // [stages] operand tile ready
 constexpr int BAR_KVE = BAR_KVF + kMaxStages;       // [stages] operand tile consumed (PV done)
-constexpr int BAR_SF = BAR_KVE + kMaxStages;        // [2] S(t) in TMEM
-constexpr int BAR_SE = BAR_SF + 2;                  // [2] S(t) read by the softmax
-constexpr int BAR_PF = BAR_SE + 2;                  // [stages] P(t) written (per stage)
+constexpr int BAR_SF = BAR_KVE + kMaxStages;        // [kNumS] S(t) in TMEM
+constexpr int BAR_SE = BAR_SF + kNumS;              // [kNumS] S(t) read by the softmax
+constexpr int BAR_PF = BAR_SE + kNumS;              // [stages] P(t) written (per stage)
 constexpr int BAR_PVD = BAR_PF + kMaxStages;        // [4] PV(t) done (by t mod 4)
 constexpr int BAR_FIN = BAR_PVD + 4;                // drain, S issuer
 constexpr int BAR_FIN2 = BAR_FIN + 1;               // drain, PV issuer
@@ -121,12 +124,13 @@ constexpr int kDsv4Page = kDsv4ScaleOff + 64 * 8;   // 37,376
 // holds 16 heads; an M=64 operand or accumulator uses lanes 0-15 or 16-31
 // of every quarter.
 //   lanes 0-15 : Q (A operand of S, bf16 packed two per column) cols [0,288)
-//                S buffers (fp32)                          cols [288,416)
+//                S buffers (fp32, 64 columns each)         cols [288,480)
 //   lanes 16-31: O (fp32, 64 heads x 512 dims)             cols [0,512)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 0;
 constexpr uint32_t kColS = 288;
 constexpr uint32_t kLaneO = 16;
+static_assert(kColS + 64u * kNumS <= kTmemCols, "S buffers fit beside the query");
 
 // Lazy rescaling: keep the running max until a new max exceeds it by more
 // than 2^8 (probabilities stay <= 256; results are unchanged).
@@ -169,7 +173,10 @@ struct Cfg {
   static constexpr int kStages = kNat ? 5 : (kConv ? 2 : 3);   // operand stages
   static constexpr int kOpBytes = kNat ? kRawTileBytes : kTileBytes;   // bytes per operand stage
   static constexpr int kRawStages = kConv ? 2 : 0;      // raw stages
-  static constexpr int kQStage = kStages - 1;           // holds the staged query until it is in TMEM (bf16 operands)
+  // the staged query (64 x d_qk bf16) sits in the last operand stage (bf16
+  // operands), or the last two (fp8: 73,728 B = two 36,864 B stages) until
+  // it is in TMEM
+  static constexpr int kQStage = kNat ? kStages - 2 : kStages - 1;
   static constexpr int kSmxWarps = kConv ? 4 : 8;
   static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + 1, kWarpIdx = kSmxWarps + 2;
   static constexpr int kWarpLoad0 = kWarpIdx + kIdxWarps;
@@ -194,7 +201,8 @@ struct Cfg {
   static constexpr int kAuxDsc = kAuxRsc + kRing * 64 * 4;   // u64  [kRing][64] DeepSeek-V4 scale blocks
   static constexpr int kAuxXch = kAuxDsc + kRing * 64 * 8;   // f32  [2][2][64] softmax exchange
   static constexpr int kAuxQsc = kAuxXch + 2 * 2 * 64 * 4;   // f32  [64] fp8 query scales
-  static constexpr int kSmemBytes = kAuxQsc + 64 * 4;
+  static constexpr int kAuxFlag = kAuxQsc + 64 * 4;          // int  [4] stream-K: last piece of the row (per quarter)
+  static constexpr int kSmemBytes = kAuxFlag + 4 * 4;
   static_assert(kSmemBytes <= 232448, "exceeds the 227 KB per-CTA shared memory of sm_100");
   static_assert(kAuxRow % 16 == 0 && kAuxRsc % 16 == 0 && kAuxDsc % 16 == 0, "aux arrays are read as vectors");
   static_assert(8 % kCopyWarps == 0 && kCpGroups >= 1 && kCpGroups <= 8, "copy-warp group ownership");
@@ -213,8 +221,11 @@ struct SplitParams {
   const int32_t* indices;      // [B, topk]
   __nv_bfloat16* out;          // [B, 64, 512]
   float* lse;                  // [B, 64]
-  float* part_o;               // [B, nsplit, 64, 512]
-  float* part_lse;             // [B, nsplit, 64]
+  float* part_o;               // [B, nsplit, 64, 512]; stream-K: [2 G, 64, 512] piece results
+  float* part_lse;             // [B, nsplit, 64]; stream-K: [2 G, 64] their lse (log2 units)
+  unsigned long long* row_ctr; // stream-K: [B, 4] arrivals per (row, lane quarter), tagged with epoch
+  unsigned long long epoch;    // stream-K: this launch's tag (1 .. 2^56 - 1)
+  int streamk;                 // 1: the G CTAs of the grid share the rows' tiles evenly (stream-K)
   int batch, topk, nsplit, ntiles_total;   // batch: decode rows (sequences x tokens)
   int tok_per_seq;             // query tokens per sequence (row b reads page-table row b / tok_per_seq)
   int cluster;                 // 1: the nsplit CTAs of a sequence form a cluster and reduce on chip
@@ -320,6 +331,11 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr)
                : "memory");
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ float ex2(float x) {
@@ -788,7 +804,9 @@ __device__ __forceinline__ void merge_tail(const float* wss, const uint4* wso, i
   }
 }
 
-template <int kKind>
+// kSK: the stream-K form (fp8 rows only), compiled apart so that the split
+// plan's kernel carries none of its row switching
+template <int kKind, bool kSK>
 __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     smla_split_kernel(const __grid_constant__ SplitParams p) {
   using C = Cfg<kKind>;
@@ -812,12 +830,30 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
   // always complete -- the staged query, the MMA drains -- keep the default)
   const long long wl = p.wait_limit;
   const int split = blockIdx.x;
-  const int b = blockIdx.y;
-  const int t_begin = (int)((long long)split * p.ntiles_total / p.nsplit);
-  const int t_end = (int)((long long)(split + 1) * p.ntiles_total / p.nsplit);
-  const int ntiles = t_end - t_begin;
-  const int tok_begin = t_begin * kTile;
-  const int tok_end = min(t_end * kTile, p.topk);
+  const int nt = p.ntiles_total;                 // 64-entry tiles per decode row
+  // This CTA's tiles: a run of the rows' tiles laid end to end in row order.
+  // Split plan: tiles [split nt / nsplit, (split + 1) nt / nsplit) of row
+  // blockIdx.y.  Stream-K plan (fp8 rows): of the W = rows x nt tiles, CTA
+  // j of the G in the grid takes [j W / G, (j + 1) W / G), which can end one
+  // row's run and begin the next; a row split between CTAs is merged by
+  // the CTA that finishes its part last.
+  constexpr bool sk = kNat && kSK;
+  int b0, tr0, ntiles;                           // first tile's row and its tile within the row
+  if (sk) {
+    const long long W = (long long)p.batch * nt;
+    const long long g0 = (long long)blockIdx.x * W / gridDim.x;
+    b0 = (int)(g0 / nt);
+    tr0 = (int)(g0 - (long long)b0 * nt);
+    ntiles = (int)((long long)(blockIdx.x + 1) * W / gridDim.x - g0);
+  } else {
+    b0 = blockIdx.y;
+    tr0 = (int)((long long)split * nt / p.nsplit);
+    ntiles = (int)((long long)(split + 1) * nt / p.nsplit) - tr0;
+  }
+  const int b = b0;                              // (split plan: the row)
+  // (split plan: every tile of the CTA lies in row b0)
+  auto tile_row = [&](int t) -> int { return sk ? b0 + (tr0 + t) / nt : b0; };
+  auto tile_in_row = [&](int t) -> int { return sk ? (tr0 + t) % nt : tr0 + t; };
 
   // The swizzled operand layouts need a 1024-byte aligned base; the dynamic
   // shared window starts there when the kernel has no static shared memory.
@@ -846,7 +882,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       mbar_init(BAR(BAR_RAW + s), kCopy + C::kBulkGroups);
       mbar_init(BAR(BAR_RAWE + s), C::kCvtWarps);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kNumS; ++s) {
       mbar_init(BAR(BAR_SF + s), 1);
       mbar_init(BAR(BAR_SE + s), kSmx);
     }
@@ -889,17 +925,18 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // once.  (Pulling the rows into L2 ahead of the loaders, one bulk
     // prefetch per row, measured slower: it queues on the copy engine.)
     auto idx_at = [&](int t, int j) -> int {
-      const int pos = tok_begin + t * kTile + j;
-      return (t < ntiles && pos < tok_end) ? __ldg(p.indices + (size_t)b * p.topk + pos) : -1;
+      if (t >= ntiles) return -1;
+      const int pos = tile_in_row(t) * kTile + j;
+      return pos < p.topk ? __ldg(p.indices + (size_t)tile_row(t) * p.topk + pos) : -1;
     };
     // An entry that names no row of the pool (past the page table, or a
     // row outside [0, num_kv_rows)) is read as padding and sets error bit 2.
-    auto row_of = [&](int idx) -> int {
+    auto row_of = [&](int idx, int drow) -> int {   // drow: the decode row of the entry
       if (idx < 0) return -1;
       long long r = idx;
       if (p.page_size) {
         if (idx >= (long long)p.pages_per_seq * p.page_size) r = -1;
-        else r = (long long)__ldg(p.page_table + (size_t)(b / p.tok_per_seq) * p.pages_per_seq + idx / p.page_size) *
+        else r = (long long)__ldg(p.page_table + (size_t)(drow / p.tok_per_seq) * p.pages_per_seq + idx / p.page_size) *
                      p.page_size +
                  idx % p.page_size;
       }
@@ -910,20 +947,22 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       return (int)r;
     };
     const int kw = warp - kWarpIdx;
-    // the 64 x kQK query (contiguous bf16) into the last operand stage,
-    // which no tile uses before the query has been moved to tensor memory
-    if (!kNat && kw == 0 && lane == 0) {
+    // the 64 x kQK query (contiguous bf16) into the last operand stage(s),
+    // which no tile uses before the query has been moved to tensor memory:
+    // one bulk copy
+    if (kw == 0 && lane == 0) {
       constexpr uint32_t kQBytes = (uint32_t)kH * kQK * 2;
       mbar_arrive_expect_tx(BAR(BAR_QS), kQBytes);
-      bulk_load_g2s(sbase + kSmemKV + C::kQStage * kTileBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
+      bulk_load_g2s(sbase + kSmemKV + C::kQStage * C::kOpBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
     }
     // Software pipeline over this warp's tiles (step S = 4), every load
     // consumed one iteration after it was issued: index of tile t+3S, page
     // entry of t+2S, row scale of t+S, then tile t is published.
     constexpr int S = kIdxWarps;
     int i2_0 = idx_at(kw + 2 * S, lane), i2_1 = idx_at(kw + 2 * S, lane + 32);                 // tile t+2S
-    int r1_0 = row_of(idx_at(kw + S, lane)), r1_1 = row_of(idx_at(kw + S, lane + 32));         // tile t+S
-    int r0_0 = row_of(idx_at(kw, lane)), r0_1 = row_of(idx_at(kw, lane + 32));                 // tile t
+    int r1_0 = row_of(idx_at(kw + S, lane), tile_row(kw + S)),                                 // tile t+S
+        r1_1 = row_of(idx_at(kw + S, lane + 32), tile_row(kw + S));
+    int r0_0 = row_of(idx_at(kw, lane), tile_row(kw)), r0_1 = row_of(idx_at(kw, lane + 32), tile_row(kw));  // tile t
     float c0_0 = 0.f, c0_1 = 0.f;                                            // scale, tile t
     uint2 d0_0 = make_uint2(0u, 0u), d0_1 = make_uint2(0u, 0u);              // scale block, tile t
     // a DeepSeek-V4 row's 8-byte scale block
@@ -952,7 +991,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         d1_0 = dsc_of(r1_0);
         d1_1 = dsc_of(r1_1);
       }
-      const int r2_0 = row_of(i2_0), r2_1 = row_of(i2_1);
+      const int r2_0 = row_of(i2_0, tile_row(t + 2 * S)), r2_1 = row_of(i2_1, tile_row(t + 2 * S));
       const int i3_0 = idx_at(t + 3 * S, lane), i3_1 = idx_at(t + 3 * S, lane + 32);
       const bool fail = t >= kRing && !mbar_wait(BAR(BAR_IXE + rs), ((t / kRing) - 1) & 1, wl);
       if (__any_sync(0xffffffffu, fail)) break;  // warp-uniform exit
@@ -1076,6 +1115,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       if constexpr (kNat) {
         if (__any_sync(0xffffffffu, t >= kStages && !mbar_wait(BAR(BAR_KVE + stage), ((t / kStages) - 1) & 1, wl)))
           break;
+        // the last two stages first hold the staged query
+        if (__any_sync(0xffffffffu, (t == C::kQStage || t == C::kQStage + 1) && !mbar_wait(BAR(BAR_QT), 0, wl)))
+          break;
         // fp8 rows as stored, into the core-matrix layout: chunk c (0..35)
         // of a row to cm_off(row in tile, c).  One instruction per row for
         // its first 512 bytes (lane = chunk), then one for the last 64 bytes
@@ -1191,15 +1233,24 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // issued, and every other warp's wait runs out in turn)
       ok = wait_all(BAR(p.stall_test ? BAR_CS1 : BAR_QT), 0);
       tc_fence_after();
+      int seg = 0;   // rows begun (stream-K)
       for (int t = 0; ok && t < ntiles; ++t) {
-        const int stage = t % kStages, sb = t & 1;
-        // S(t) reuses the S buffer of S(t-2): its softmax must have read it.
-        // (Nothing else orders S(t) after PV(t-2): issued as soon as the
-        // softmax has read S(t-2), S(t) is done by the time the softmax
-        // reaches tile t, which measured faster than holding it behind
-        // PV(t-2).)
-        if (t >= 2) {
-          ok = wait_all(BAR(BAR_SE + sb), ((t >> 1) - 1) & 1);
+        const int stage = t % kStages, sb = t % kNumS;
+        if (sk && t > 0 && tile_in_row(t) == 0) {
+          // tile t begins the next row: its query replaces the last one in
+          // tensor memory (written once the last row's scores were read)
+          ++seg;
+          ok = wait_all(BAR(BAR_QT), (uint32_t)(seg & 1));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        // S(t) reuses the S buffer of S(t-kNumS): its softmax must have read
+        // it.  (Nothing else orders S(t) after the PV MMAs before it: issued
+        // as soon as its buffer is free, S(t) is done by the time the
+        // softmax reaches tile t, which measured faster than holding it
+        // behind PV(t-2).)
+        if (t >= kNumS) {
+          ok = wait_all(BAR(BAR_SE + sb), ((t / kNumS) - 1) & 1);
           if (!ok) break;
           tc_fence_after();
         }
@@ -1237,6 +1288,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         ok = wait_all(BAR(BAR_PF + stage), (t / kStages) & 1);
         if (!ok) break;
         tc_fence_after();
+        const bool fresh = t == 0 || (sk && tile_in_row(t) == 0);   // O starts over (a row's first tile)
         if constexpr (kNat) {
           // O[:, 256 hf + n] += P8[:, 32 kk + k] V[32 (kk mod 2) + k, 256 hf + n]:
           // A = P buffer t mod 4 (codes 0-63: high parts of the 64 tokens,
@@ -1251,7 +1303,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
             for (int hf = 0; hf < 2; ++hf) {
               const uint64_t bb = cm_desc(vb + (uint32_t)(((4 * (kk & 1)) * (kRawRowBytes / 16) + 16 * hf) * 128),
                                           kCmGroupBytes, 128);
-              mma8_ss_elect(o0 + 256u * (uint32_t)hf, dp + (uint64_t)(2 * kk), bb, kIdescPV8, t > 0 || kk > 0);
+              mma8_ss_elect(o0 + 256u * (uint32_t)hf, dp + (uint64_t)(2 * kk), bb, kIdescPV8, !fresh || kk > 0);
             }
           }
         } else {
@@ -1268,7 +1320,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
               const uint32_t d = o0 + 256u * (uint32_t)hf;
               const uint64_t a = dp + (uint64_t)(2 * kk);
               const uint64_t bb = bv + (uint64_t)(128 * kk + 2048 * hf);
-              if (t == 0 && kk == 0) mma_set_elect(d, a, bb, kIdescPV);
+              if (fresh && kk == 0) mma_set_elect(d, a, bb, kIdescPV);
               else mma_acc_elect(d, a, bb, kIdescPV);
             }
           }
@@ -1317,54 +1369,66 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // fp8: 2^-sq, the power of two the head's query was scaled by
     float q_unscale = 1.f;
     bool aborted = false;
-    if constexpr (kNat) {
-      float* s_qsc = reinterpret_cast<float*>(smem + C::kAuxQsc);
-      if (u == 0) {
-        // The query row as e4m3 parts in tensor memory: x = q * 2^sq (the
-        // head's largest |q| scaled into [128, 256)), high part e4m3(x) at
-        // columns [0, 144), low part e4m3(x - high) at [144, 288); this
-        // thread's dims [288 half, +288) are columns [72 half, +72) of each.
-        // Read straight from global memory, twice (the scale first).
-        const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((size_t)b * kH + h) * (kDqk * 2) + half * kDqk);
-        uint32_t amax = 0;   // largest |q| as bf16 magnitude bits (ordered like the values)
+    float* s_qsc = reinterpret_cast<float*>(smem + C::kAuxQsc);
+    // fp8 (warps u == 0): decode row r's query into tensor memory as e4m3
+    // parts: x = q * 2^sq (the head's largest |q| scaled into [128, 256)),
+    // high part e4m3(x) at columns [0, 144), low part e4m3(x - high) at
+    // [144, 288); this thread's dims [288 half, +288) are columns
+    // [72 half, +72) of each.  Read twice (the scale first) from the copy
+    // staged in shared memory (the CTA's first row), or else straight from
+    // global memory.  Then the scale goes to s_qsc for the quarter's other
+    // warp and the warp arrives on BAR_QT.
+    auto load_query = [&](int r, bool staged) {
+      const uint4* qg = reinterpret_cast<const uint4*>(p.q + ((size_t)r * kH + h) * (kDqk * 2) + half * kDqk);
+      const uint32_t qs = sbase + kSmemKV + C::kQStage * C::kOpBytes + (uint32_t)(h * (kDqk * 2) + half * kDqk);
+      auto q16 = [&](int k4) -> uint4 { return staged ? ld_shared_v4(qs + 16u * (uint32_t)k4) : __ldg(qg + k4); };
+      uint32_t amax = 0;   // largest |q| as bf16 magnitude bits (ordered like the values)
 #pragma unroll 4
-        for (int k4 = 0; k4 < kDqk / 16; ++k4) {
-          const uint4 v = __ldg(qg + k4);
+      for (int k = 0; k < kDqk / 16; ++k) {
+        // (staged: lane-rotated order, so that the half-warp's 16 head
+        // rows, 1152 bytes apart, meet in different banks)
+        const int k4 = staged ? (k + lane) % (kDqk / 16) : k;
+        const uint4 v = q16(k4);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) amax = max(amax, max(w4[k] & 0x7FFFu, (w4[k] >> 16) & 0x7FFFu));
+      }
+      amax = max(amax, (uint32_t)__shfl_xor_sync(0xffffffffu, (int)amax, 16));
+      const float qmax = __uint_as_float(amax << 16);
+      const int sq = qmax > 0.f ? min(126, max(-126, 7 - ilog2f(qmax))) : 0;   // (subnormal maxima: 126)
+      const float qscale = pow2i(sq);
+      q_unscale = pow2i(-sq);
+#pragma unroll 1
+      for (int c = 0; c < kDqk / 64; ++c) {   // 32 dims per step
+        uint32_t hw[8], lw[8];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const uint4 v = q16(4 * c + k4);
           const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) amax = max(amax, max(w4[k] & 0x7FFFu, (w4[k] >> 16) & 0x7FFFu));
-        }
-        amax = max(amax, (uint32_t)__shfl_xor_sync(0xffffffffu, (int)amax, 16));
-        const float qmax = __uint_as_float(amax << 16);
-        const int sq = qmax > 0.f ? min(126, max(-126, 7 - ilog2f(qmax))) : 0;   // (subnormal maxima: 126)
-        const float qscale = pow2i(sq);
-        q_unscale = pow2i(-sq);
-#pragma unroll 1
-        for (int c = 0; c < kDqk / 64; ++c) {   // 32 dims per step
-          uint32_t hw[8], lw[8];
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const uint4 v = __ldg(qg + 4 * c + k4);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int k = 0; k < 4; k += 2) {
-              uint32_t h0, l0, h1, l1;
-              split_e4m3x2(__uint_as_float(w4[k] << 16) * qscale, __uint_as_float(w4[k] & 0xFFFF0000u) * qscale,
-                           h0, l0);
-              split_e4m3x2(__uint_as_float(w4[k + 1] << 16) * qscale,
-                           __uint_as_float(w4[k + 1] & 0xFFFF0000u) * qscale, h1, l1);
-              hw[2 * k4 + k / 2] = h0 | (h1 << 16);
-              lw[2 * k4 + k / 2] = l0 | (l1 << 16);
-            }
+          for (int k = 0; k < 4; k += 2) {
+            uint32_t h0, l0, h1, l1;
+            split_e4m3x2(__uint_as_float(w4[k] << 16) * qscale, __uint_as_float(w4[k] & 0xFFFF0000u) * qscale,
+                         h0, l0);
+            split_e4m3x2(__uint_as_float(w4[k + 1] << 16) * qscale,
+                         __uint_as_float(w4[k + 1] & 0xFFFF0000u) * qscale, h1, l1);
+            hw[2 * k4 + k / 2] = h0 | (h1 << 16);
+            lw[2 * k4 + k / 2] = l0 | (l1 << 16);
           }
-          tmem_st_16x32bx2_x8<72>(tmem + q_lanes + kColQ + 8u * (uint32_t)c, hw);
-          tmem_st_16x32bx2_x8<72>(tmem + q_lanes + kColQ + 144u + 8u * (uint32_t)c, lw);
         }
-        tmem_wait_st();
-        if (lane < 16) s_qsc[h] = q_unscale;
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(BAR_QT));
+        tmem_st_16x32bx2_x8<72>(tmem + q_lanes + kColQ + 8u * (uint32_t)c, hw);
+        tmem_st_16x32bx2_x8<72>(tmem + q_lanes + kColQ + 144u + 8u * (uint32_t)c, lw);
+      }
+      tmem_wait_st();
+      if (lane < 16) s_qsc[h] = q_unscale;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(BAR_QT));
+    };
+    if constexpr (kNat) {
+      if (u == 0) {
+        if (!mbar_wait(BAR(BAR_QS), 0)) aborted = true;
+        load_query(b0, true);
       } else {
         // the other warp of the quarter takes the head's scale once the
         // query is in place
@@ -1400,10 +1464,212 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // fp8: O and its normaliser are kept times sig2 (0 until the first
     // nonzero probability), the power of two of the e4m3 P parts
     float sig2 = 0.f;
-    const float fsc = p.scale_log2 * q_unscale;
+    float fsc = p.scale_log2 * q_unscale;
+    // stream-K: the row being computed, its first tile here, rows begun
+    int srow = b0, sfirst = 0, seg = 0;
+    // both warps of the quarter (the named barrier of the pair)
+    auto pair_sync = [&]() {
+      if constexpr (kU == 2) named_bar_sync(2 + q, 64);
+      else __syncwarp();
+    };
+    // Stream-K: row r's result from this CTA's tiles [t0, t1).  A row that
+    // lies wholly in this CTA is written out straight from tensor memory.
+    // Otherwise each of the CTAs that hold part of it (a piece) counts
+    // itself in at the row's counter (one per lane quarter, so the quarters
+    // never wait for one another); the last piece to arrive merges: every
+    // other piece has left its result, normalised, and its lse in its slot
+    // (slot 2 j for the first row of CTA j, 2 j + 1 for its last), and the
+    // last piece adds them to its own, weighted by 2^(lse - max), as the
+    // log-sum-exp combine does.  No CTA waits for another.  The counter
+    // holds (epoch << 8) | arrivals; a tag other than this launch's reads as
+    // zero arrivals, and the last piece sets it back to 0, so the workspace
+    // needs no initialisation.
+    auto finish_row = [&](int r, int t0, int t1) {
+      if (!aborted) {
+        // PV(t1-2) then PV(t1-1): each wait is at most one phase ahead
+        if (t1 - t0 >= 2 && !mbar_wait(BAR(BAR_PVD + ((t1 - 2) & 3)), ((t1 - 2) >> 2) & 1, wl)) aborted = true;
+        if (!mbar_wait(BAR(BAR_PVD + ((t1 - 1) & 3)), ((t1 - 1) >> 2) & 1, wl)) aborted = true;
+        tc_fence_after();
+      }
+      float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      l_tot = pair_reduce(l_tot, false, aborted);
+      if (aborted) return;
+      const float l_nrm = l_tot * sig2;
+      const float inv_l = l_tot > 0.f && l_nrm > 0.f ? 1.f / l_nrm : 0.f;
+      const float lse2 = l_tot > 0.f ? m_run + log2f(l_tot) : -INFINITY;   // log2 units
+      const long long W = (long long)p.batch * nt;
+      const long long G = gridDim.x;
+      auto owner = [&](long long g) -> int { return (int)(((g + 1) * G - 1) / W); };   // CTA of global tile g
+      const int j0 = owner((long long)r * nt), j1 = owner((long long)(r + 1) * nt - 1);
+      __nv_bfloat16* orow = p.out + ((size_t)r * kH + h) * kDv;
+      if (j0 == j1) {
+#pragma unroll 1
+        for (int c = kOc * u; c < kOc * (u + 1); ++c) {
+          float o[32];
+          tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
+          tmem_wait_ld();
+          uint4* dst = reinterpret_cast<uint4*>(orow + half * 256 + c * 32);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            dst[k4] = make_uint4(pack_bf16x2(o[8 * k4] * inv_l, o[8 * k4 + 1] * inv_l),
+                                 pack_bf16x2(o[8 * k4 + 2] * inv_l, o[8 * k4 + 3] * inv_l),
+                                 pack_bf16x2(o[8 * k4 + 4] * inv_l, o[8 * k4 + 5] * inv_l),
+                                 pack_bf16x2(o[8 * k4 + 6] * inv_l, o[8 * k4 + 7] * inv_l));
+        }
+        if (u == 0 && half == 0) p.lse[(size_t)r * kH + h] = lse2 * 0.6931471805599453f;
+        return;
+      }
+      const unsigned npc = (unsigned)(j1 - j0 + 1);
+      const unsigned long long ep = p.epoch;
+      unsigned long long* ctr = p.row_ctr + (size_t)r * 4 + q;
+      int* s_flag = reinterpret_cast<int*>(smem + C::kAuxFlag);
+      // 1. has every other piece arrived already?  Then this one merges
+      //    without leaving its own result.
+      if (u == 0 && lane == 0) {
+        const unsigned long long v = ld_relaxed_gpu_u64(ctr);
+        const unsigned c = (v >> 8) == ep ? (unsigned)(v & 255u) : 0u;
+        const int lastp = c + 1 == npc;
+        if (lastp) {
+          __threadfence();
+          atomicExch(ctr, 0ull);
+        }
+        s_flag[q] = lastp;
+      }
+      pair_sync();
+      bool last = s_flag[q] != 0;
+      if (!last) {
+        // 2. this piece's result (normalised) and lse to its slot, then
+        //    count it in
+        const int slot = 2 * (int)blockIdx.x + (r == b0 ? 0 : 1);
+        float* so = p.part_o + ((size_t)slot * kH + h) * kDv;
+#pragma unroll 1
+        for (int c = kOc * u; c < kOc * (u + 1); ++c) {
+          float o[32];
+          tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
+          tmem_wait_ld();
+          float4* dst = reinterpret_cast<float4*>(so + half * 256 + c * 32);
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4)
+            dst[k4] = make_float4(__fmul_rn(o[4 * k4], inv_l), __fmul_rn(o[4 * k4 + 1], inv_l),
+                                  __fmul_rn(o[4 * k4 + 2], inv_l), __fmul_rn(o[4 * k4 + 3], inv_l));
+        }
+        if (u == 0 && half == 0) p.part_lse[(size_t)slot * kH + h] = lse2;
+        __threadfence();
+        pair_sync();
+        if (u == 0 && lane == 0) {
+          unsigned long long v = ld_relaxed_gpu_u64(ctr);
+          int lastp = -1;
+          // (each failed exchange is another piece's arrival: at most npc - 1)
+          for (int it = 0; it < 64; ++it) {
+            const unsigned c = (v >> 8) == ep ? (unsigned)(v & 255u) : 0u;
+            const unsigned long long nv = c + 1 == npc ? 0ull : ((ep << 8) | (unsigned long long)(c + 1));
+            const unsigned long long pv = atomicCAS(ctr, v, nv);
+            if (pv == v) {
+              lastp = c + 1 == npc ? 1 : 0;
+              break;
+            }
+            v = pv;
+          }
+          if (lastp < 0) atomicOr(&g_error_word, 1u);
+          if (lastp == 1) __threadfence();
+          s_flag[q] = lastp == 1;
+        }
+        pair_sync();
+        last = s_flag[q] != 0;
+      }
+      if (!last) return;
+      // 3. merge, in the order of the pieces (CTA j0 first) whichever
+      //    merges, so the result does not depend on the order of arrival:
+      //    the pieces' lse and weights, then per 32-dim chunk their
+      //    normalised results (from L2; this piece's from tensor memory,
+      //    normalised as it would have been stored) weighted and summed
+      //    with one rounding per product and per sum
+      const int self = (int)blockIdx.x;
+      float lk[kMaxPieces];
+      const float* po[kMaxPieces];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < kMaxPieces; ++k) {
+        const int j = j0 + k;
+        lk[k] = -INFINITY;
+        po[k] = nullptr;
+        if (j == self) {
+          lk[k] = lse2;
+        } else if (j <= j1) {
+          const long long first_g = (long long)j * W / G;   // CTA j's first tile
+          const int sl = 2 * j + (first_g / nt == r ? 0 : 1);
+          lk[k] = __ldcg(p.part_lse + (size_t)sl * kH + h);
+          po[k] = p.part_o + ((size_t)sl * kH + h) * kDv + half * 256;
+        }
+        mx = fmaxf(mx, lk[k]);
+      }
+      float wk[kMaxPieces], wsum = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxPieces; ++k) {
+        wk[k] = lk[k] == -INFINITY ? 0.f : ex2(lk[k] - mx);
+        wsum = __fadd_rn(wsum, wk[k]);
+      }
+      const float inv_w = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll 1
+      for (int c = kOc * u; c < kOc * (u + 1); ++c) {
+        float o[32];
+        tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
+        tmem_wait_ld();
+        uint4* dst = reinterpret_cast<uint4*>(orow + half * 256 + c * 32);
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {   // 8 dims at a time
+          float acc[8];
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) acc[e2] = 0.f;
+#pragma unroll
+          for (int k = 0; k < kMaxPieces; ++k) {
+            const float f = __fmul_rn(wk[k], inv_w);
+            if (j0 + k == self) {
+#pragma unroll
+              for (int e2 = 0; e2 < 8; ++e2)
+                acc[e2] = __fadd_rn(acc[e2], __fmul_rn(f, __fmul_rn(o[8 * g8 + e2], inv_l)));
+            } else if (po[k] != nullptr) {
+              const float4* src = reinterpret_cast<const float4*>(po[k] + c * 32 + 8 * g8);
+              const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
+              const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+              for (int e2 = 0; e2 < 8; ++e2) acc[e2] = __fadd_rn(acc[e2], __fmul_rn(f, v[e2]));
+            }
+          }
+          dst[g8] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                               pack_bf16x2(acc[6], acc[7]));
+        }
+      }
+      if (u == 0 && half == 0)
+        p.lse[(size_t)r * kH + h] = wsum > 0.f ? (mx + log2f(wsum)) * 0.6931471805599453f : -INFINITY;
+    };
     for (int i = 0; i < ntiles; ++i) {
-      const int sb = i & 1, rs = i % kRing;
-      if (!mbar_wait(BAR(BAR_SF + sb), (i >> 1) & 1, wl) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1, wl))
+      if (sk && i > 0 && tile_in_row(i) == 0) {
+        // Tile i begins the next row.  The quarter's two warps agree to go
+        // on; the next row's query goes to tensor memory first (the last
+        // row's scores have all been read, and the next row's first scores
+        // are then computed during this epilogue), then the last row's
+        // result is written and the running state starts over.
+        if constexpr (kU == 2) aborted = group_any(aborted, 2 + q, 64);
+        else aborted = __any_sync(0xffffffffu, aborted);
+        if (aborted) break;
+        ++seg;
+        if (u == 0) load_query(srow + 1, false);
+        finish_row(srow, sfirst, i);
+        if (u != 0) {
+          if (!mbar_wait(BAR(BAR_QT), (uint32_t)(seg & 1), wl)) aborted = true;
+          q_unscale = s_qsc[h];
+        }
+        m_run = -INFINITY;
+        l_run = 0.f;
+        l_pv = 0.f;
+        sig2 = 0.f;
+        fsc = p.scale_log2 * q_unscale;
+        ++srow;
+        sfirst = i;
+      }
+      const int sb = i % kNumS, rs = i % kRing;
+      if (!mbar_wait(BAR(BAR_SF + sb), (i / kNumS) & 1, wl) || !mbar_wait(BAR(BAR_IXS + rs), (i / kRing) & 1, wl))
         aborted = true;
       aborted = __any_sync(0xffffffffu, aborted);
       float s[kTok];
@@ -1591,85 +1857,89 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     // this CTA's tiles are done: the next kernel of the stream may start
     // on idle SMs (it waits for this grid's completion before reading)
     if (threadIdx.x == 0) grid_dep_launch();
-    if (!aborted && ntiles > 0) {
-      // PV(n-2) then PV(n-1): each wait is at most one phase ahead
-      if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + ((ntiles - 2) & 3)), ((ntiles - 2) >> 2) & 1, wl)) aborted = true;
-      if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 3)), ((ntiles - 1) >> 2) & 1, wl)) aborted = true;
-      tc_fence_after();
-    }
-    // the head's totals over its kU warps (and the common abort decision)
-    float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
-    l_tot = pair_reduce(l_tot, false, aborted);
-    // the normaliser of O (bf16 operands: the rounded-P sum; fp8: the
-    // probability sum times sig2) and the split's weight in a merge (the
-    // rounded-P sum; fp8: the probability sum)
-    float l_w = l_tot;
-    if constexpr (!kNat) {
-      l_w = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
-      l_w = pair_reduce(l_w, false, aborted);
-    }
-    const float l_nrm = kNat ? l_tot * sig2 : l_w;
-    if (p.cluster) {
-      // in-cluster merge (after the warp roles): this split's per-head
-      // statistics (max, merge weight, fp32 sum) go to the workspace
-      merge_failed = aborted;
-      if (!aborted && u == 0 && half == 0) {
-        float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * kStatFloats;
-        *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * kStatFloats) = make_float4(m_run, l_w, l_tot, 0.f);
-        // for the merge writers: 1 / (normaliser of O) of head h
-        reinterpret_cast<float*>(smem + C::kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
+    if (sk) {
+      if (ntiles > 0) finish_row(srow, sfirst, ntiles);
+    } else {
+      if (!aborted && ntiles > 0) {
+        // PV(n-2) then PV(n-1): each wait is at most one phase ahead
+        if (ntiles >= 2 && !mbar_wait(BAR(BAR_PVD + ((ntiles - 2) & 3)), ((ntiles - 2) >> 2) & 1, wl)) aborted = true;
+        if (!mbar_wait(BAR(BAR_PVD + ((ntiles - 1) & 3)), ((ntiles - 1) >> 2) & 1, wl)) aborted = true;
+        tc_fence_after();
       }
-    } else if (!aborted) {
-      const bool any = l_tot > 0.f;
-      const float inv_l = any && l_nrm > 0.f ? 1.f / l_nrm : 0.f;
-      const float lse_h = any ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
-      const bool direct = p.nsplit == 1;
-      const size_t part = (size_t)b * p.nsplit + split;
-      // Stage the head rows in shared memory (the idle operand stages) with
-      // a 16-byte pad per row, which makes the 16-byte stores of a warp
-      // conflict-free, then write each row with one bulk copy.
-      const uint32_t row_bytes = direct ? kDv * 2 : kDv * 4;
-      const uint32_t stride = row_bytes + 16;
-      uint8_t* srow = smem + kSmemKV + (size_t)h * stride;
-#pragma unroll 1
-      for (int c = kOc * u; c < kOc * (u + 1); ++c) {
-        float o[32];
-        if (ntiles > 0) {
-          tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0.f;
-        }
-        const int d0 = half * 256 + c * 32;   // this thread's 32 dims
-        if (direct) {
-          uint4* dst = reinterpret_cast<uint4*>(srow + d0 * 2);
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            dst[k4] = make_uint4(pack_bf16x2(o[8 * k4] * inv_l, o[8 * k4 + 1] * inv_l),
-                                 pack_bf16x2(o[8 * k4 + 2] * inv_l, o[8 * k4 + 3] * inv_l),
-                                 pack_bf16x2(o[8 * k4 + 4] * inv_l, o[8 * k4 + 5] * inv_l),
-                                 pack_bf16x2(o[8 * k4 + 6] * inv_l, o[8 * k4 + 7] * inv_l));
-        } else {
-          float4* dst = reinterpret_cast<float4*>(srow + d0 * 4);
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4)
-            dst[k4] = make_float4(o[4 * k4] * inv_l, o[4 * k4 + 1] * inv_l, o[4 * k4 + 2] * inv_l,
-                                  o[4 * k4 + 3] * inv_l);
-        }
+      // the head's totals over its kU warps (and the common abort decision)
+      float l_tot = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+      l_tot = pair_reduce(l_tot, false, aborted);
+      // the normaliser of O (bf16 operands: the rounded-P sum; fp8: the
+      // probability sum times sig2) and the split's weight in a merge (the
+      // rounded-P sum; fp8: the probability sum)
+      float l_w = l_tot;
+      if constexpr (!kNat) {
+        l_w = l_pv + __shfl_xor_sync(0xffffffffu, l_pv, 16);
+        l_w = pair_reduce(l_w, false, aborted);
       }
-      fence_proxy_async_smem();
-      // the row's other chunks come from the other warp of the quarter
-      if constexpr (kU == 2) named_bar_sync(2 + q, 64);
-      else __syncwarp();
-      if (u == 0 && half == 0) {
-        uint8_t* gdst = direct ? reinterpret_cast<uint8_t*>(p.out + ((size_t)b * kH + h) * kDv)
-                               : reinterpret_cast<uint8_t*>(p.part_o + (part * kH + h) * kDv);
-        bulk_store_s2g(gdst, smem_u32(srow), row_bytes);
-        bulk_commit();
-        if (direct) p.lse[(size_t)b * kH + h] = lse_h;
-        else p.part_lse[part * kH + h] = lse_h;
-        bulk_wait_all();
+      const float l_nrm = kNat ? l_tot * sig2 : l_w;
+      if (p.cluster) {
+        // in-cluster merge (after the warp roles): this split's per-head
+        // statistics (max, merge weight, fp32 sum) go to the workspace
+        merge_failed = aborted;
+        if (!aborted && u == 0 && half == 0) {
+          float* wss = p.part_lse + (size_t)b * p.nsplit * 64 * kStatFloats;
+          *reinterpret_cast<float4*>(wss + ((size_t)split * 64 + h) * kStatFloats) = make_float4(m_run, l_w, l_tot, 0.f);
+          // for the merge writers: 1 / (normaliser of O) of head h
+          reinterpret_cast<float*>(smem + C::kAuxRow)[h] = l_nrm > 0.f ? 1.f / l_nrm : 0.f;
+        }
+      } else if (!aborted) {
+        const bool any = l_tot > 0.f;
+        const float inv_l = any && l_nrm > 0.f ? 1.f / l_nrm : 0.f;
+        const float lse_h = any ? (m_run + log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
+        const bool direct = p.nsplit == 1;
+        const size_t part = (size_t)b * p.nsplit + split;
+        // Stage the head rows in shared memory (the idle operand stages) with
+        // a 16-byte pad per row, which makes the 16-byte stores of a warp
+        // conflict-free, then write each row with one bulk copy.
+        const uint32_t row_bytes = direct ? kDv * 2 : kDv * 4;
+        const uint32_t stride = row_bytes + 16;
+        uint8_t* srow = smem + kSmemKV + (size_t)h * stride;
+  #pragma unroll 1
+        for (int c = kOc * u; c < kOc * (u + 1); ++c) {
+          float o[32];
+          if (ntiles > 0) {
+            tmem_ld_16x32bx2_x32_h256(tmem + o_lanes + 32u * (uint32_t)c, o);
+            tmem_wait_ld();
+          } else {
+  #pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = 0.f;
+          }
+          const int d0 = half * 256 + c * 32;   // this thread's 32 dims
+          if (direct) {
+            uint4* dst = reinterpret_cast<uint4*>(srow + d0 * 2);
+  #pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              dst[k4] = make_uint4(pack_bf16x2(o[8 * k4] * inv_l, o[8 * k4 + 1] * inv_l),
+                                   pack_bf16x2(o[8 * k4 + 2] * inv_l, o[8 * k4 + 3] * inv_l),
+                                   pack_bf16x2(o[8 * k4 + 4] * inv_l, o[8 * k4 + 5] * inv_l),
+                                   pack_bf16x2(o[8 * k4 + 6] * inv_l, o[8 * k4 + 7] * inv_l));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(srow + d0 * 4);
+  #pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4)
+              dst[k4] = make_float4(o[4 * k4] * inv_l, o[4 * k4 + 1] * inv_l, o[4 * k4 + 2] * inv_l,
+                                    o[4 * k4 + 3] * inv_l);
+          }
+        }
+        fence_proxy_async_smem();
+        // the row's other chunks come from the other warp of the quarter
+        if constexpr (kU == 2) named_bar_sync(2 + q, 64);
+        else __syncwarp();
+        if (u == 0 && half == 0) {
+          uint8_t* gdst = direct ? reinterpret_cast<uint8_t*>(p.out + ((size_t)b * kH + h) * kDv)
+                                 : reinterpret_cast<uint8_t*>(p.part_o + (part * kH + h) * kDv);
+          bulk_store_s2g(gdst, smem_u32(srow), row_bytes);
+          bulk_commit();
+          if (direct) p.lse[(size_t)b * kH + h] = lse_h;
+          else p.part_lse[part * kH + h] = lse_h;
+          bulk_wait_all();
+        }
       }
     }
     tc_fence_before();
@@ -1872,7 +2142,7 @@ static smla_status validate_shape(const smla_shape* s) {
   if (s->tokens_per_seq < 0 || s->tokens_per_seq > 16 || (long long)s->batch * tokens_of(s) > 65535)
     return SMLA_ERR_INVALID_ARG;
   if (s->num_kv_rows < 1 || s->num_kv_rows > 0x7FFFFFFFLL) return SMLA_ERR_INVALID_ARG;
-  if (s->nsplit < 0) return SMLA_ERR_INVALID_ARG;
+  if (s->nsplit < 0 && s->nsplit != SMLA_NSPLIT_STREAMK) return SMLA_ERR_INVALID_ARG;
   if (s->kv_dtype != SMLA_KV_BF16 && s->kv_dtype != SMLA_KV_FP8_E4M3_ROWSCALE && s->kv_dtype != SMLA_KV_DSV4_PAGED)
     return SMLA_ERR_UNSUPPORTED;
   const int want_qk = s->kv_dtype == SMLA_KV_DSV4_PAGED ? 512 : kDqk;
@@ -1899,7 +2169,7 @@ static int device_sm_count() {
 static int plan_nsplit_raw(const smla_shape* s, int num_sms) {
   const int tiles = (s->topk + kTile - 1) / kTile;
   int n;
-  if (s->nsplit > 0) {
+  if (s->nsplit > 0) {      // (SMLA_NSPLIT_STREAMK without a stream-K plan: automatic)
     n = s->nsplit;
   } else {
     n = num_sms > 0 ? num_sms / rows_of(s) : 1;
@@ -1916,13 +2186,29 @@ static int plan_nsplit_raw(const smla_shape* s, int num_sms) {
 // nsplit is kept as given (merged in the kernel whenever it can launch as a
 // cluster); an automatic plan takes the largest such n that fits in one
 // wave (falling back to one split).
+//
+// Stream-K (asked for with nsplit = SMLA_NSPLIT_STREAMK): fp8 rows with
+// lists of at least 16 tiles, more rows than half the SMs but not a multiple
+// of them, are shared out over one CTA per SM: the rows' tiles are laid end
+// to end and each CTA takes an equal run (so a row falls to at most three
+// CTAs), merged inside the kernel by the CTA that finishes its part of the
+// row last.  Other shapes asking for it get the automatic plan.
 struct Plan {
   int n;
   bool cluster;
+  bool streamk;
 };
-static Plan make_plan(const smla_shape* s, int num_sms, const int active[5]) {
-  Plan pl{plan_nsplit_raw(s, num_sms), false};
-  if (pl.n < 2) return pl;
+static bool streamk_fits(const smla_shape* s, int num_sms) {
+  if (s->kv_dtype != SMLA_KV_FP8_E4M3_ROWSCALE || s->nsplit != SMLA_NSPLIT_STREAMK || num_sms < 2) return false;
+  const long long rows = rows_of(s), nt = (s->topk + kTile - 1) / kTile;
+  return nt >= 16 && 2 * rows > num_sms && rows % num_sms != 0 && rows * nt < (1ll << 31);
+}
+static Plan make_plan(const smla_shape* s, int num_sms, const int active[5], bool allow_streamk = true) {
+  Plan pl{plan_nsplit_raw(s, num_sms), false, false};
+  if (pl.n < 2) {
+    pl.streamk = allow_streamk && streamk_fits(s, num_sms);
+    return pl;
+  }
   if (s->nsplit > 0) {
     if ((pl.n & (pl.n - 1)) == 0 && pl.n <= 16) pl.cluster = active[31 - __builtin_clz(pl.n)] >= 1;
     return pl;
@@ -1932,9 +2218,9 @@ static Plan make_plan(const smla_shape* s, int num_sms, const int active[5]) {
   // best split count for every batch and list length tried.
   for (int lg = 4; lg >= 1; --lg) {
     const int c = 1 << lg;
-    if (c <= pl.n && active[lg] >= rows_of(s)) return Plan{c, true};
+    if (c <= pl.n && active[lg] >= rows_of(s)) return Plan{c, true, false};
   }
-  return Plan{1, false};
+  return Plan{1, false, false};
 }
 
 static size_t partial_bytes(int batch, int nsplit) {
@@ -1955,18 +2241,36 @@ static size_t workspace_bytes_for(int batch, int nsplit, bool cluster) {
   if (nsplit < 2) return 0;
   return cluster ? cluster_bytes(batch, nsplit) : partial_bytes(batch, nsplit);
 }
+// Workspace of a stream-K plan over a grid of g CTAs: two result slots per
+// CTA (its first and last row, when another CTA shares them) as fp32
+// [2 g, 64, 512], their lse [2 g, 64], then the row counters [rows, 4] u64.
+static size_t streamk_o_bytes(int g) { return (((size_t)2 * g * kH * kDv * 4) + 255) / 256 * 256; }
+static size_t streamk_lse_bytes(int g) { return (((size_t)2 * g * kH * 4) + 255) / 256 * 256; }
+static size_t streamk_bytes(int rows, int g) {
+  return streamk_o_bytes(g) + streamk_lse_bytes(g) + (((size_t)rows * 4 * 8) + 255) / 256 * 256;
+}
+static size_t plan_workspace_bytes(const smla_shape* s, const Plan& pl, int num_sms) {
+  return pl.streamk ? streamk_bytes(rows_of(s), num_sms) : workspace_bytes_for(rows_of(s), pl.n, pl.cluster);
+}
+// A tag per launch for the stream-K row counters (never 0, below 2^56).
+static unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> counter{0};
+  unsigned long long e = 0;
+  while (e == 0) e = (counter.fetch_add(1) + 1) & ((1ull << 56) - 1);
+  return e;
+}
 
 // The shared-memory opt-in is set once per device (an idempotent call, so a
 // race between threads is harmless); later calls, including calls made
 // while a stream is being captured into a CUDA graph, skip it.
-template <int kKind>
+template <int kKind, bool kSK = false>
 static cudaError_t ensure_smem_attr() {
   static volatile int done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-  const cudaError_t e =
-      cudaFuncSetAttribute(smla_split_kernel<kKind>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<kKind>::kSmemBytes);
+  const cudaError_t e = cudaFuncSetAttribute(smla_split_kernel<kKind, kSK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Cfg<kKind>::kSmemBytes);
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
   return e;
 }
@@ -1987,7 +2291,7 @@ static const ClusterCaps& cluster_caps() {
   if (done[dev]) return cache[dev];
   ClusterCaps caps = {{0, 0, 0, 0, 0}};
   if (ensure_smem_attr<kKind>() == cudaSuccess &&
-      cudaFuncSetAttribute(smla_split_kernel<kKind>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+      cudaFuncSetAttribute(smla_split_kernel<kKind, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
           cudaSuccess) {
     for (int lg = 1; lg <= 4; ++lg) {
       cudaLaunchAttribute at[1];
@@ -2002,7 +2306,7 @@ static const ClusterCaps& cluster_caps() {
       cfg.attrs = at;
       cfg.numAttrs = 1;
       int k = 0;
-      if (cudaOccupancyMaxActiveClusters(&k, smla_split_kernel<kKind>, &cfg) == cudaSuccess) caps.active[lg] = k;
+      if (cudaOccupancyMaxActiveClusters(&k, smla_split_kernel<kKind, false>, &cfg) == cudaSuccess) caps.active[lg] = k;
     }
   }
   cudaGetLastError();  // a refused query leaves no sticky error
@@ -2017,10 +2321,17 @@ static const ClusterCaps& caps_for(const smla_shape* s) {
 }
 
 template <int kKind>
-static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
-  auto kern = smla_split_kernel<kKind>;
+static cudaError_t launch_split(const SplitParams& prm, int grid_x, cudaStream_t stream) {
+  auto kern = smla_split_kernel<kKind, false>;
   cudaError_t e = ensure_smem_attr<kKind>();
   if (e != cudaSuccess) return e;
+  if constexpr (kKind == kKindFp8) {
+    if (prm.streamk) {
+      kern = smla_split_kernel<kKind, true>;
+      e = ensure_smem_attr<kKind, true>();
+      if (e != cudaSuccess) return e;
+    }
+  }
   // programmatic dependent launch (the kernel waits for its prerequisites
   // itself), and for an in-cluster merge the cluster of nsplit CTAs
   cudaLaunchAttribute at[2];
@@ -2036,7 +2347,7 @@ static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
     ++na;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(prm.nsplit, prm.batch);
+  cfg.gridDim = prm.streamk ? dim3(grid_x, 1) : dim3(prm.nsplit, prm.batch);
   cfg.blockDim = dim3(Cfg<kKind>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg<kKind>::kSmemBytes;
   cfg.stream = stream;
@@ -2048,7 +2359,7 @@ static cudaError_t launch_split(const SplitParams& prm, cudaStream_t stream) {
 static smla_status run_split(const smla_shape* shape, const void* q, const void* kv_cache,
                              const float* kv_row_scale, const int32_t* page_table, const int32_t* indices,
                              float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                             int32_t* nsplit_out, cudaStream_t stream, int* nsplit_used, bool allow_cluster,
+                             int32_t* nsplit_out, cudaStream_t stream, int* nsplit_used, bool allow_fused,
                              bool* cluster_used, long long wait_limit = kWaitLimitCycles, int stall_test = 0) {
   smla_status st = validate_shape(shape);
   if (st != SMLA_OK) return st;
@@ -2062,12 +2373,14 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   if (!(scale == scale) || isinf(scale)) return SMLA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   if (sms <= 0) return SMLA_ERR_CUDA;
-  const Plan pl = make_plan(shape, sms, caps_for(shape).active);
+  // (allow_fused: the in-kernel merges, in a cluster or stream-K, may be used)
+  const Plan pl = make_plan(shape, sms, caps_for(shape).active, allow_fused);
   const int n = pl.n;
-  const bool cluster = allow_cluster && pl.cluster;
-  if (n > 1) {
+  const bool cluster = allow_fused && pl.cluster;
+  if (n > 1 || pl.streamk) {
     if (!workspace || !aligned(workspace, 256)) return SMLA_ERR_WORKSPACE;
-    if (workspace_bytes < workspace_bytes_for(rows_of(shape), n, cluster)) return SMLA_ERR_WORKSPACE;
+    const size_t need = pl.streamk ? streamk_bytes(rows_of(shape), sms) : workspace_bytes_for(rows_of(shape), n, cluster);
+    if (workspace_bytes < need) return SMLA_ERR_WORKSPACE;
   }
   SplitParams prm;
   memset(&prm, 0, sizeof(prm));
@@ -2094,9 +2407,17 @@ static smla_status run_split(const smla_shape* shape, const void* q, const void*
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634);
   prm.wait_limit = wait_limit;
   prm.stall_test = stall_test;
-  const cudaError_t e = fp8 ? launch_split<kKindFp8>(prm, stream)
-                            : (shape->kv_dtype == SMLA_KV_DSV4_PAGED ? launch_split<kKindDsv4>(prm, stream)
-                                                                    : launch_split<kKindBf16>(prm, stream));
+  if (pl.streamk) {
+    prm.streamk = 1;
+    prm.epoch = next_epoch();
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    prm.part_o = reinterpret_cast<float*>(ws);
+    prm.part_lse = reinterpret_cast<float*>(ws + streamk_o_bytes(sms));
+    prm.row_ctr = reinterpret_cast<unsigned long long*>(ws + streamk_o_bytes(sms) + streamk_lse_bytes(sms));
+  }
+  const cudaError_t e = fp8 ? launch_split<kKindFp8>(prm, sms, stream)
+                            : (shape->kv_dtype == SMLA_KV_DSV4_PAGED ? launch_split<kKindDsv4>(prm, sms, stream)
+                                                                    : launch_split<kKindBf16>(prm, sms, stream));
   if (e != cudaSuccess) return SMLA_ERR_CUDA;
   if (nsplit_out) *nsplit_out = n;
   if (nsplit_used) *nsplit_used = n;
@@ -2194,13 +2515,15 @@ int32_t sparse_mla_plan_nsplit(const smla_shape* shape) {
 
 size_t sparse_mla_workspace_size(const smla_shape* shape) {
   if (smla::validate_shape(shape) != SMLA_OK) return 0;
-  const smla::Plan pl = smla::make_plan(shape, smla::device_sm_count(), smla::caps_for(shape).active);
-  return smla::workspace_bytes_for(smla::rows_of(shape), pl.n, pl.cluster);
+  const int sms = smla::device_sm_count();
+  const smla::Plan pl = smla::make_plan(shape, sms, smla::caps_for(shape).active);
+  return smla::plan_workspace_bytes(shape, pl, sms);
 }
 
 int32_t sparse_mla_plan_merge(const smla_shape* shape) {
   if (smla::validate_shape(shape) != SMLA_OK) return -1;
   const smla::Plan pl = smla::make_plan(shape, smla::device_sm_count(), smla::caps_for(shape).active);
+  if (pl.streamk) return 3;
   return pl.n < 2 ? 0 : (pl.cluster ? 1 : 2);
 }
 
@@ -2259,7 +2582,8 @@ smla_status sparse_mla_decode_static_scratch(const smla_shape* shape, const void
   }
   const int sms = smla::device_sm_count();
   if (sms <= 0) return SMLA_ERR_CUDA;
-  const smla::Plan pl = smla::make_plan(shape, sms, smla::caps_for(shape).active);
+  // (the split plan: a stream-K plan's workspace is larger than the scratch)
+  const smla::Plan pl = smla::make_plan(shape, sms, smla::caps_for(shape).active, false);
   const int n = pl.n;
   const size_t need = smla::workspace_bytes_for(smla::rows_of(shape), n, pl.cluster);
   if (need > SMLA_STATIC_SCRATCH_BYTES) return SMLA_ERR_WORKSPACE;

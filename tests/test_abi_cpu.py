@@ -84,7 +84,7 @@ INVALID, UNSUPPORTED = 1, 2
 
 @pytest.mark.parametrize("kw,code", [
     (dict(batch=0), INVALID), (dict(batch=70000), INVALID), (dict(topk=0), INVALID),
-    (dict(num_kv_rows=0), INVALID), (dict(nsplit=-1), INVALID),
+    (dict(num_kv_rows=0), INVALID), (dict(nsplit=-2), INVALID),
     # multi-token decode: 0..16 tokens per sequence, at most 65535 decode rows
     (dict(tokens_per_seq=-1), INVALID), (dict(tokens_per_seq=17), INVALID),
     (dict(batch=5000, tokens_per_seq=16), INVALID),
