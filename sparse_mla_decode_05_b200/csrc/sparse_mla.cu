@@ -157,11 +157,11 @@ constexpr long long kWaitLimitCycles = 4000000000ll;
 
 // Warp roles: S softmax/epilogue warps (two per tensor-memory lane quarter,
 // or one for DeepSeek-V4 caches), then the S-MMA issuer (+ TMEM allocator),
-// the PV-MMA issuer, four index resolvers (resolver k owns the tiles t = k
-// mod 4), the copy warps and, for DeepSeek-V4 caches, eight warps that
-// convert the raw codes to bf16 operand tiles.  The in-cluster merge uses
-// warps 0-7 and, for the lse, warps 8-9, all done with their roles by then.
-constexpr int kIdxWarps = 4;
+// the PV-MMA issuer, the index resolvers (four, or two for fp8 rows:
+// resolver k owns the tiles t = k mod their count), the copy warps and, for
+// DeepSeek-V4 caches, eight warps that convert the raw codes to bf16 operand
+// tiles.  The in-cluster merge uses warps 0-7 and, for the lse, warps 8-9,
+// all done with their roles by then.
 // cache layouts the split kernel is instantiated for
 constexpr int kKindBf16 = 0;   // bf16 rows [N, 576]
 constexpr int kKindFp8 = 1;    // e4m3fn rows [N, 576] + one fp32 scale per row
@@ -179,6 +179,10 @@ struct Cfg {
   static constexpr int kQStage = kNat ? kStages - 2 : kStages - 1;
   static constexpr int kSmxWarps = kConv ? 4 : 8;
   static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + 1, kWarpIdx = kSmxWarps + 2;
+  // fp8: two resolvers (16 warps in all, 128 registers a thread) measured
+  // ~2 % faster on 2048-entry lists; bf16 operands keep four (two were ~4 %
+  // slower on 512-entry lists)
+  static constexpr int kIdxWarps = kNat ? 2 : 4;
   static constexpr int kWarpLoad0 = kWarpIdx + kIdxWarps;
   static constexpr int kCopyWarps = kConv ? 2 : 4;
   static constexpr int kCvtWarps = kConv ? 8 : 0;
@@ -917,13 +921,14 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + C::kAuxTmem);
 
   bool merge_failed = false;   // a softmax warp gave up (in-cluster merge)
-  if (warp >= kWarpIdx && warp < kWarpIdx + kIdxWarps) {
+  if (warp >= kWarpIdx && warp < kWarpIdx + C::kIdxWarps) {
     // ------------------------------------------------------------ index warps
     // Resolve each tile's 64 entries to physical rows (and fp8 row scales)
-    // into the kRing-deep ring ahead of the loaders.  Warp k handles tiles
-    // t = k, k+4, ... (ring slot k), so four tiles' lookups are in flight at
-    // once.  (Pulling the rows into L2 ahead of the loaders, one bulk
-    // prefetch per row, measured slower: it queues on the copy engine.)
+    // into the kRing-deep ring ahead of the loaders.  Warp k of the S =
+    // kIdxWarps handles tiles t = k, k+S, ... (ring slot t mod kRing), and
+    // each keeps three tiles' lookups in flight.  (Pulling the rows into L2
+    // ahead of the loaders, one bulk prefetch per row, measured slower: it
+    // queues on the copy engine.)
     auto idx_at = [&](int t, int j) -> int {
       if (t >= ntiles) return -1;
       const int pos = tile_in_row(t) * kTile + j;
@@ -955,10 +960,10 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       mbar_arrive_expect_tx(BAR(BAR_QS), kQBytes);
       bulk_load_g2s(sbase + kSmemKV + C::kQStage * C::kOpBytes, p.q + (size_t)b * kQBytes, kQBytes, BAR(BAR_QS));
     }
-    // Software pipeline over this warp's tiles (step S = 4), every load
+    // Software pipeline over this warp's tiles (step S), every load
     // consumed one iteration after it was issued: index of tile t+3S, page
     // entry of t+2S, row scale of t+S, then tile t is published.
-    constexpr int S = kIdxWarps;
+    constexpr int S = C::kIdxWarps;
     int i2_0 = idx_at(kw + 2 * S, lane), i2_1 = idx_at(kw + 2 * S, lane + 32);                 // tile t+2S
     int r1_0 = row_of(idx_at(kw + S, lane), tile_row(kw + S)),                                 // tile t+S
         r1_1 = row_of(idx_at(kw + S, lane + 32), tile_row(kw + S));
