@@ -113,7 +113,10 @@ constexpr int BAR_IXE = BAR_IXS + kRing;            // [kRing] rows consumed
 constexpr int BAR_RAW = BAR_IXE + kRing;            // [raw stages] raw rows landed
 constexpr int BAR_RAWE = BAR_RAW + kMaxStages;      // [raw stages] raw rows converted
 constexpr int BAR_CS1 = BAR_RAWE + kMaxStages;      // cluster: every split's blocks written
-constexpr int kNumBars = BAR_CS1 + 1;
+constexpr int BAR_SH = BAR_CS1 + 1;                 // [kNumS] S(t) high part done (split S issue)
+constexpr int BAR_FIN3 = BAR_SH + kNumS;            // drain, second S issuer
+constexpr int BAR_FIN4 = BAR_FIN3 + 1;              // drain, second PV issuer
+constexpr int kNumBars = BAR_FIN4 + 1;
 // DeepSeek-V4 page: 64 slots of 576 bytes (448 e4m3fn codes, 64 bf16), then
 // 64 scale blocks of 8 bytes (7 UE8M0 exponents, one per 64 code dims)
 constexpr int kDsv4Slot = 576, kDsv4Nope = 448;
@@ -178,7 +181,17 @@ struct Cfg {
   // it is in TMEM
   static constexpr int kQStage = kNat ? kStages - 2 : kStages - 1;
   static constexpr int kSmxWarps = kConv ? 4 : 8;
-  static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + 1, kWarpIdx = kSmxWarps + 2;
+  // MMA issuers.  fp8: four, one per SM sub-partition (warp w runs on
+  // sub-partition w mod 4): S(t) is issued in two halves, the query's high
+  // part by kWarpS and then, once that has completed, its low part by
+  // kWarpS2 (18 MMAs each), and PV(t) by kWarpPV (dims 0-255) and kWarpPV2
+  // (256-511).  A warp issuing a long run of MMAs slows the softmax warps
+  // of its own sub-partition, which then hold up every PV; spread over the
+  // four sub-partitions this measured faster than two issuers.
+  static constexpr bool kSplitIss = kNat;
+  static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + 1;
+  static constexpr int kWarpS2 = kSplitIss ? kSmxWarps + 2 : -1, kWarpPV2 = kSplitIss ? kSmxWarps + 3 : -1;
+  static constexpr int kWarpIdx = kSmxWarps + (kSplitIss ? 4 : 2);
   // fp8: two resolvers (16 warps in all, 128 registers a thread) measured
   // ~2 % faster on 2048-entry lists; bf16 operands keep four (two were ~4 %
   // slower on 512-entry lists)
@@ -877,7 +890,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       // bf16: one arrival per copying thread (when its copies land); fp8 /
       // DeepSeek-V4: one per convert warp
       mbar_init(BAR(BAR_KVF + s), kConv ? C::kCvtWarps : kCopy);
-      mbar_init(BAR(BAR_KVE + s), 1);
+      mbar_init(BAR(BAR_KVE + s), C::kSplitIss ? 2 : 1);   // one commit per PV issuer
       mbar_init(BAR(BAR_PF + s), kSmx);
     }
     for (int s = 0; s < C::kRawStages; ++s) {
@@ -890,9 +903,12 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       mbar_init(BAR(BAR_SF + s), 1);
       mbar_init(BAR(BAR_SE + s), kSmx);
     }
-    for (int s = 0; s < 4; ++s) mbar_init(BAR(BAR_PVD + s), 1);
+    for (int s = 0; s < 4; ++s) mbar_init(BAR(BAR_PVD + s), C::kSplitIss ? 2 : 1);
+    for (int s = 0; s < kNumS; ++s) mbar_init(BAR(BAR_SH + s), 1);
     mbar_init(BAR(BAR_FIN), 1);
     mbar_init(BAR(BAR_FIN2), 1);
+    mbar_init(BAR(BAR_FIN3), 1);
+    mbar_init(BAR(BAR_FIN4), 1);
     mbar_init(BAR(BAR_QT), 4);
     mbar_init(BAR(BAR_QS), 1);
     mbar_init(BAR(BAR_CS1), p.cluster ? p.nsplit : 1);
@@ -1219,19 +1235,36 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       }
     }
     cp_async_wait_all();
-  } else if (warp == kWarpS || warp == kWarpPV) {
+  } else if (warp == kWarpS || warp == kWarpPV || warp == C::kWarpS2 || warp == C::kWarpPV2) {
     // ------------------------------------------------------------ MMA issuers
-    // Two warps issue tensor-core work, each blocking (in hardware) on one
-    // barrier at a time: warp kWarpS computes S(t) once tile t has landed;
-    // warp kWarpPV computes PV(t) once P(t) is written.  Each warp runs with
-    // warp-uniform state and one elected lane issues; tcgen05.commit tracks
-    // the issuing thread's own MMAs.  Operand addresses advance by constants
-    // (shared descriptors: byte offset >> 4; tensor memory: columns).
+    // Warps that issue tensor-core work, each blocking (in hardware) on one
+    // barrier at a time: warp kWarpS computes S(t) once tile t has landed
+    // (fp8: its first half, then kWarpS2 the second once the first has
+    // completed); warp kWarpPV computes PV(t) once P(t) is written (fp8:
+    // dims 0-255, kWarpPV2 dims 256-511).  Each warp runs with warp-uniform
+    // state and one elected lane issues; tcgen05.commit tracks the issuing
+    // thread's own MMAs.  Operand addresses advance by constants (shared
+    // descriptors: byte offset >> 4; tensor memory: columns).
     auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
       return __shfl_sync(0xffffffffu, (int)mbar_wait(bar, parity, wl), 0) != 0;
     };
     bool ok = true;
-    if (warp == kWarpS) {
+    if (C::kSplitIss && warp == C::kWarpS2) {
+      // the second half of S(t): the query's low part (K steps 18-35),
+      // accumulated once the high part has completed
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int stage = t % kStages, sb = t % kNumS;
+        ok = wait_all(BAR(BAR_SH + sb), (t / kNumS) & 1);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tmem + kColS + 64u * (uint32_t)sb;
+        const uint64_t bk = cm_desc(sbase + kSmemKV + stage * C::kOpBytes, 128, kCmGroupBytes);
+#pragma unroll
+        for (int k = kDqk / 32; k < 2 * kDqk / 32; ++k)
+          mma8_ts_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + (uint64_t)((k % 18) * 16), kIdescS8, true);
+        commit_elect(BAR(BAR_SF + sb));
+      }
+    } else if (warp == kWarpS) {
       const uint64_t dk0 = sw128_desc(sbase + kSmemKV, 16, 1024);
       // (stall_test: the cluster barrier, which nothing arrives on without a
       // cluster, stands in for the query: the wait runs out, no MMA is
@@ -1264,12 +1297,13 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
         const uint32_t d = tmem + kColS + 64u * (uint32_t)sb;
         if constexpr (kNat) {
           // 36 K steps of 32 codes: the query's high part (steps 0-17), then
-          // its low part (18-35), each against K chunks 2 (k mod 18) and +1
-          // (+256 B, +16 in the descriptor); Q columns +8 per step
+          // its low part (18-35, issued by kWarpS2), each against K chunks
+          // 2 (k mod 18) and +1 (+256 B, +16 in the descriptor); Q columns +8
+          // per step
           const uint64_t bk = cm_desc(sbase + kSmemKV + stage * C::kOpBytes, 128, kCmGroupBytes);
           mma8_ts_elect(d, tmem + kColQ, bk, kIdescS8, false);
 #pragma unroll
-          for (int k = 1; k < 2 * kDqk / 32; ++k)
+          for (int k = 1; k < (C::kSplitIss ? 1 : 2) * kDqk / 32; ++k)
             mma8_ts_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + (uint64_t)((k % 18) * 16), kIdescS8, true);
         } else {
           // stage s starts s * kTileBytes later (descriptor address field: bytes >> 4)
@@ -1283,10 +1317,12 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
             mma_ts_acc_elect(d, tmem + kColQ + 8u * (uint32_t)k, bk + off, kIdescS);
           }
         }
-        commit_elect(BAR(BAR_SF + sb));
+        commit_elect(BAR((C::kSplitIss ? BAR_SH : BAR_SF) + sb));
       }
     } else {
       const uint64_t dv0 = sw128_desc(sbase + kSmemKV, kAtomBytes, 1024);
+      // (fp8: this warp's half of the output dims)
+      const int hf0 = C::kSplitIss && warp == C::kWarpPV2 ? 1 : 0, hf1 = C::kSplitIss ? hf0 + 1 : 2;
       const uint32_t o0 = tmem + (kLaneO << 16);
       for (int t = 0; ok && t < ntiles; ++t) {
         const int stage = t % kStages;
@@ -1305,7 +1341,7 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            for (int hf = hf0; hf < hf1; ++hf) {
               const uint64_t bb = cm_desc(vb + (uint32_t)(((4 * (kk & 1)) * (kRawRowBytes / 16) + 16 * hf) * 128),
                                           kCmGroupBytes, 128);
               mma8_ss_elect(o0 + 256u * (uint32_t)hf, dp + (uint64_t)(2 * kk), bb, kIdescPV8, !fresh || kk > 0);
@@ -1335,8 +1371,9 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
       }
     }
     // drain: every MMA this warp issued has completed before teardown
-    commit_elect(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2));
-    mbar_wait(BAR(warp == kWarpS ? BAR_FIN : BAR_FIN2), 0);
+    const int fin = warp == kWarpS ? BAR_FIN : warp == kWarpPV ? BAR_FIN2 : warp == C::kWarpS2 ? BAR_FIN3 : BAR_FIN4;
+    commit_elect(BAR(fin));
+    mbar_wait(BAR(fin), 0);
   } else if (warp < kSmx) {
     // ------------------------------------------------------------ softmax
     // kSmx warps; warp w reaches tensor-memory lane quarter q = w % 4 (heads
@@ -1979,8 +2016,8 @@ __global__ void __launch_bounds__(Cfg<kKind>::kThreads, 1)
     float* wss = p.part_lse + (size_t)b * n * 64 * kStatFloats;  // [src][64][8]: m, l_pv, l, -, part scales
     bool failed = merge_failed;
     if (upper) {
-      // every PV has completed (the PV issuer's drain barrier: one phase)
-      failed = !mbar_wait(BAR(BAR_FIN2), 0);
+      // every PV has completed (the PV issuers' drain barriers: one phase)
+      failed = !mbar_wait(BAR(BAR_FIN2), 0) || (C::kSplitIss && !mbar_wait(BAR(BAR_FIN4), 0));
       tc_fence_after();
     }
     const bool bad = group_any(failed, 1, 256);
