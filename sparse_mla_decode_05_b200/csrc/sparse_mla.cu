@@ -187,17 +187,23 @@ struct Cfg {
   // kWarpS2 (18 MMAs each), and PV(t) by kWarpPV (dims 0-255) and kWarpPV2
   // (256-511).  A warp issuing a long run of MMAs slows the softmax warps
   // of its own sub-partition, which then hold up every PV; spread over the
-  // four sub-partitions this measured faster than two issuers.
+  // four sub-partitions this measured faster than two issuers (c5: 73.4 ->
+  // 68.0 us).  With two copy warps (below) each sub-partition holds two
+  // softmax warps, one issuer and an index or a copy warp; the S halves
+  // beside the index warps (warps 8, 9) and the PV halves beside the copy
+  // warps (10, 11) measured best of the placements tried.
   static constexpr bool kSplitIss = kNat;
-  static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + 1;
-  static constexpr int kWarpS2 = kSplitIss ? kSmxWarps + 2 : -1, kWarpPV2 = kSplitIss ? kSmxWarps + 3 : -1;
+  static constexpr int kWarpS = kSmxWarps, kWarpPV = kSmxWarps + (kSplitIss ? 2 : 1);
+  static constexpr int kWarpS2 = kSplitIss ? kSmxWarps + 1 : -1, kWarpPV2 = kSplitIss ? kSmxWarps + 3 : -1;
   static constexpr int kWarpIdx = kSmxWarps + (kSplitIss ? 4 : 2);
   // fp8: two resolvers (16 warps in all, 128 registers a thread) measured
   // ~2 % faster on 2048-entry lists; bf16 operands keep four (two were ~4 %
   // slower on 512-entry lists)
   static constexpr int kIdxWarps = kNat ? 2 : 4;
   static constexpr int kWarpLoad0 = kWarpIdx + kIdxWarps;
-  static constexpr int kCopyWarps = kConv ? 2 : 4;
+  // copy warps: fp8 rows two (16 warps in all, four per sub-partition:
+  // c5 66.7 -> 62.7 us against four), bf16 rows four
+  static constexpr int kCopyWarps = kConv || kNat ? 2 : 4;
   static constexpr int kCvtWarps = kConv ? 8 : 0;
   static constexpr int kCopyThreads = kCopyWarps * 32;
   static constexpr int kLoadWarps = kCopyWarps + kCvtWarps;
