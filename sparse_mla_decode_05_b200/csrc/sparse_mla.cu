@@ -14,18 +14,19 @@
 //  * Gather each top-k KV tile ONCE and reuse it for all 64 heads, instead of
 //    one program per head re-reading the same rows 64 times ([Diag] "The
 //    Subject Message"; [Design] "Design Decisions" 1).  Here one CTA owns
-//    (sequence, top-k chunk); 64-token tiles are gathered into shared memory
-//    with 16-byte cp.async (fp8 rows: codes copied, then converted exactly
-//    to bf16 in shared memory) and consumed by the tensor cores for every
-//    head.
+//    (decode row, top-k chunk); 64-token tiles are gathered into shared
+//    memory with 16-byte cp.async and consumed by the tensor cores for every
+//    head (fp8 rows as stored; DeepSeek-V4 pages through convert warps).
 //  * Scores and PV as tensor-core contractions across the head group with
 //    fp32 accumulation ([Design] "Design Decisions" 5-6).  Here: tcgen05.mma
 //    with accumulators in tensor memory (TMEM):
 //        S  = Q . K^T   M = 64 heads, N = 64 tokens, K = 576, Q read from TMEM
 //        O += P . V     M = 64 heads, N = 2 x 256 dims, K = 64 tokens
-//    The query sits in tensor memory and three 64-row tiles in shared
-//    memory: B200's 227 KB per CTA lets BLOCK_H = 64 (all heads) fit, which
-//    the pages' ~99 KB sm_120 budget forbade ([Design] "Memory Budgeting").
+//    (kind::f16 for bf16 rows; kind::f8f6f4 on the fp8 codes, with the
+//    query and P as exact e4m3 high + low parts).  The query sits in tensor
+//    memory and several 64-row tiles in shared memory: B200's 227 KB per CTA
+//    lets BLOCK_H = 64 (all heads) fit, which the pages' ~99 KB sm_120
+//    budget forbade ([Design] "Memory Budgeting").
 //  * Online softmax in fp32; masked entries (index -1) take no part
 //    ([Design] "Edge Case Handling").  Rows of masked entries are zero-filled
 //    in shared memory and their probabilities are exactly 0.
@@ -35,12 +36,11 @@
 //    CUDA-graph capture ([Truth] "The Split-K Solution: Reasoning About the
 //    Fix"; [Pivot] "The Reasoning: Weighing Two Paths").
 //
-// Warp roles in the split kernel (one CTA per SM; ~227 KB shared memory):
-//   warps 0-3  softmax + epilogue (128 threads; warp w owns TMEM lanes 32w..)
-//   warp  4    TMEM allocator; issues S = Q K^T
-//   warp  5    issues O += P V
-//   warps 6-9  resolve indices (flat or paged) to rows
-//   warps 10.. gather rows (and, for fp8 codes, convert them)
+// Warp roles in the split kernel (one CTA per SM; ~223-227 KB shared
+// memory), set per cache kind by Cfg below: softmax + epilogue warps (two per
+// TMEM lane quarter; one for DeepSeek-V4 pages), the MMA issuers (S and PV;
+// fp8: four, one per SM sub-partition), the index resolvers, the copy warps
+// and, for DeepSeek-V4 pages, the convert warps.
 // Every wait on a pipeline barrier is bounded (about 2 s): on expiry the CTA
 // records an error bit in a device word, drains its own copies and MMAs,
 // frees TMEM and exits.
